@@ -1,0 +1,343 @@
+"""Pins for the CPU oracle: each check comes from something other than the
+oracle itself (a hand-derived fixture, a library routine, a closed form, an
+invariant, planted structure, or brute force written as plain loops)."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import minf_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "masks_small.txt")
+
+
+def _golden_cases():
+    cases = {}
+    name = None
+    for line in open(GOLDEN):
+        line = line.rstrip("\n")
+        if not line or line.startswith("#"):
+            continue
+        if line.startswith("case "):
+            parts = line.split()
+            name = parts[1]
+            params = dict(p.split("=") for p in parts[2:])
+            cases[name] = (params, [])
+        else:
+            cases[name][1].append([int(t) for t in line.split()])
+    return cases
+
+
+def _to_mask(rows_lists, N):
+    m = np.zeros((len(rows_lists), N), bool)
+    for i, js in enumerate(rows_lists):
+        m[i, js] = True
+    return m
+
+
+# ----------------------------------------------------------------- masks
+
+def test_golden_ashape_mask():
+    p, rows = _golden_cases()["ashape"]
+    N = int(p["N"])
+    got = orc.mask_ashape(np.arange(N), N, int(p["n_sink"]), int(p["n_local"]))
+    assert np.array_equal(got, _to_mask(rows, N))
+
+
+def test_golden_vs_mask():
+    p, rows = _golden_cases()["vs"]
+    N, blk = int(p["N"]), int(p["block"])
+    V = [int(x) for x in p["V"].split(",")]
+    S = [int(x) for x in p["S"].split(",")]
+    got = orc.mask_vs(np.arange(N), N, V, S, block=blk)
+    assert np.array_equal(got, _to_mask(rows, N))
+
+
+def test_golden_bs_mask():
+    p, rows = _golden_cases()["bs"]
+    N, blk = int(p["N"]), int(p["block"])
+    sels = [[int(x) for x in p[f"sel{b}"].split(",")] for b in range(N // blk)]
+    k = max(len(s) for s in sels)
+    idx = np.full((len(sels), k), -1)
+    for b, s in enumerate(sels):
+        idx[b, :len(s)] = s
+    cnt = np.array([len(s) for s in sels])
+    got = orc.mask_bs(np.arange(N), N, idx, cnt, block=blk)
+    assert np.array_equal(got, _to_mask(rows, N))
+
+
+@pytest.mark.parametrize("N", [64, 192, 320])
+def test_masks_reduce_to_causal(N):
+    """All-selected closed forms: every pattern with everything kept is causal."""
+    rows = np.arange(N)
+    dense = np.tril(np.ones((N, N), bool))
+    assert np.array_equal(orc.mask_dense(rows, N), dense)
+    assert np.array_equal(orc.mask_ashape(rows, N, 0, N), dense)
+    assert np.array_equal(orc.mask_ashape(rows, N, N, 1), dense)
+    assert np.array_equal(orc.mask_vs(rows, N, np.arange(N), [0]), dense)
+    assert np.array_equal(orc.mask_vs(rows, N, [], np.arange(N)), dense)
+    nb = N // 64
+    idx = np.tile(np.arange(nb), (nb, 1))
+    cnt = np.arange(1, nb + 1)
+    idx = np.where(np.arange(nb)[None, :] < cnt[:, None], idx, -1)
+    assert np.array_equal(orc.mask_bs(rows, N, idx, cnt), dense)
+
+
+def test_vs_mask_offset0_is_block_diagonal_causal():
+    N = 256
+    m = orc.mask_vs(np.arange(N), N, [], [0])
+    i, j = np.meshgrid(np.arange(N), np.arange(N), indexing="ij")
+    assert np.array_equal(m, (j <= i) & (i // 64 == j // 64))
+
+
+def test_vs_mask_covers_exact_diagonals():
+    """Every element on a selected diagonal (i - j = o) lies in the mask."""
+    rng = np.random.default_rng(3)
+    N = 512
+    S = np.unique(np.concatenate([[0], rng.choice(N, 20, replace=False)]))
+    V = np.unique(rng.choice(N, 12, replace=False))
+    m = orc.mask_vs(np.arange(N), N, V, S)
+    for o in S:
+        i = np.arange(o, N)
+        assert m[i, i - o].all()
+    for j in V:
+        assert m[np.arange(j, N), j].all()
+    assert not m[np.triu_indices(N, 1)].any()
+
+
+# ------------------------------------------------------------- attention
+
+def _sdpa_ref(q, k, v):
+    qt = torch.from_numpy(q)[None, None]
+    kt = torch.from_numpy(k)[None, None]
+    vt = torch.from_numpy(v)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)[0, 0].numpy()
+
+
+@pytest.mark.parametrize("N,d", [(37, 8), (200, 16), (257, 32)])
+def test_dense_attention_matches_library(N, d):
+    rng = np.random.default_rng(N)
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    O, L = orc.attention_head(q, k, v, np.arange(N), lambda r: orc.mask_dense(r, N),
+                              orc.default_scale(d))
+    assert np.allclose(O, _sdpa_ref(q, k, v), atol=1e-12, rtol=1e-10)
+    s = (q @ k.T) / math.sqrt(d)
+    from scipy.special import logsumexp
+    ref_lse = np.array([logsumexp(s[i, :i + 1]) for i in range(N)])
+    assert np.allclose(L, ref_lse, atol=1e-12)
+
+
+def test_masked_attention_bruteforce_loops():
+    """Arbitrary mask vs plain Python loops (math.exp), including an empty row."""
+    rng = np.random.default_rng(11)
+    N, d = 12, 3
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    mask = rng.random((N, N)) < 0.5
+    mask[4] = False
+    scale = 0.7
+    O, L = orc.attention_rows(q, k, v, mask, scale)
+    for i in range(N):
+        js = [j for j in range(N) if mask[i, j]]
+        if not js:
+            assert np.all(O[i] == 0) and L[i] == -np.inf
+            continue
+        s = [scale * sum(q[i, t] * k[j, t] for t in range(d)) for j in js]
+        mx = max(s)
+        w = [math.exp(x - mx) for x in s]
+        tot = sum(w)
+        for t in range(d):
+            ref = sum(w[a] * v[js[a], t] for a in range(len(js))) / tot
+            assert abs(O[i, t] - ref) < 1e-12
+        assert abs(L[i] - (mx + math.log(tot))) < 1e-12
+
+
+def test_sparse_with_all_indices_equals_dense():
+    """Closed form: VS with every column (and BS with every block) is dense causal."""
+    rng = np.random.default_rng(5)
+    N, d = 256, 16
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    sc = orc.default_scale(d)
+    rows = np.arange(N)
+    Od, Ld = orc.attention_head(q, k, v, rows, lambda r: orc.mask_dense(r, N), sc)
+    V, S = orc.vs_select(*orc.vs_estimate(q[-64:], k, sc), N, N)
+    Ov, Lv = orc.attention_head(q, k, v, rows, lambda r: orc.mask_vs(r, N, V, S), sc)
+    assert np.allclose(Ov, Od, atol=1e-12) and np.allclose(Lv, Ld, atol=1e-12)
+    idx, cnt = orc.bs_select(q, k, sc, N // 64)
+    Ob, Lb = orc.attention_head(q, k, v, rows, lambda r: orc.mask_bs(r, N, idx, cnt), sc)
+    assert np.allclose(Ob, Od, atol=1e-12) and np.allclose(Lb, Ld, atol=1e-12)
+
+
+# ------------------------------------------------------- VS estimation
+
+def test_vs_estimate_bruteforce_loops():
+    rng = np.random.default_rng(2)
+    N, L, d = 40, 8, 4
+    q, k = rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    scale = 0.5
+    v, sg = orc.vs_estimate(q[N - L:], k, scale, row_chunk=3)
+    vr = [0.0] * N
+    sr = [0.0] * N
+    for i in range(N - L, N):
+        s = [scale * sum(q[i, t] * k[j, t] for t in range(d)) for j in range(i + 1)]
+        mx = max(s)
+        e = [math.exp(x - mx) for x in s]
+        tot = sum(e)
+        for j in range(i + 1):
+            vr[j] += e[j] / tot
+            sr[i - j] += e[j] / tot
+    assert np.allclose(v, vr, atol=1e-13) and np.allclose(sg, sr, atol=1e-13)
+
+
+def test_vs_estimate_mass_closed_form():
+    """Each of the L rows is a probability distribution: both score vectors sum to L."""
+    rng = np.random.default_rng(4)
+    N, d = 1000, 32
+    q, k = rng.standard_normal((64, d)), rng.standard_normal((N, d))
+    v, sg = orc.vs_estimate(q, k, 1 / math.sqrt(d))
+    assert abs(v.sum() - 64) < 1e-9 and abs(sg.sum() - 64) < 1e-9
+    assert (v >= 0).all() and (sg >= 0).all()
+    # the last row sees every key: column N-1 only gets that row's mass
+    assert v[N - 1] < 1.0
+
+
+def test_vs_planted_column_and_diagonal():
+    rng = np.random.default_rng(9)
+    N, d = 1024, 32
+    q = rng.standard_normal((N, d))
+    k = 0.05 * rng.standard_normal((N, d))
+    u = q[N - 64:].mean(axis=0)
+    j_star = 137
+    k[j_star] = 6.0 * u / np.linalg.norm(u) * math.sqrt(d)
+    V, _ = orc.vs_select(*orc.vs_estimate(q[N - 64:], k, 1 / math.sqrt(d)), 1, 1)
+    assert V.tolist() == [j_star]
+
+    o_star = 300
+    k2 = 0.05 * rng.standard_normal((N, d))
+    k2[: N - o_star] = 1.5 * q[o_star:]          # k_j aligned with q_{j + o*}
+    v2, s2 = orc.vs_estimate(q[N - 64:], k2, 1 / math.sqrt(d))
+    _, S = orc.vs_select(v2, s2, 1, 2)
+    assert S.tolist() == [0, o_star]
+
+
+# ------------------------------------------------------------ selection
+
+@pytest.mark.parametrize("seed", range(6))
+def test_select_topk_equals_full_sort(seed):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(1, 300))
+    scores = rng.integers(0, 12, n).astype(np.float64)       # many ties
+    k = int(rng.integers(1, n + 3))
+    forced = int(rng.integers(0, n)) if seed % 2 else None
+    got = orc.select_topk(scores, k, forced=forced)
+    key = [(-(math.inf if j == forced else scores[j]), j) for j in range(n)]
+    ref = sorted(j for _, j in sorted(key)[:min(k, n)])
+    assert got.tolist() == ref
+
+
+def test_select_topk_rows_matches_rowwise():
+    rng = np.random.default_rng(1)
+    R, C, k = 40, 40, 7
+    scores = rng.integers(-5, 5, (R, C)).astype(np.float64)
+    valid = np.arange(C)[None, :] <= np.arange(R)[:, None]
+    idx, cnt = orc.select_topk_rows(scores, valid, k, forced_col=np.arange(R))
+    for r in range(R):
+        ref = orc.select_topk(scores[r, : r + 1], k, forced=r)
+        assert cnt[r] == min(k, r + 1)
+        assert idx[r, : cnt[r]].tolist() == ref.tolist()
+        assert (idx[r, cnt[r]:] == -1).all()
+
+
+# ------------------------------------------------------- BS estimation
+
+def test_bs_pool_loops():
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((256, 5))
+    p = orc.bs_pool(x)
+    for b in range(4):
+        for t in range(5):
+            assert abs(p[b, t] - sum(x[64 * b + r, t] for r in range(64)) / 64) < 1e-14
+
+
+def test_bs_select_planted_and_forced_diagonal():
+    rng = np.random.default_rng(8)
+    N, d = 64 * 16, 16
+    q = rng.standard_normal((N, d))
+    k = rng.standard_normal((N, d))
+    dirn = rng.standard_normal(d)
+    q[64 * 12: 64 * 13] += 4 * dirn                 # query block 12
+    k[64 * 3: 64 * 4] += 4 * dirn                   # key block 3
+    idx, cnt = orc.bs_select(q, k, 1 / math.sqrt(d), 2)
+    assert idx[12].tolist() == [3, 12]
+    nb = N // 64
+    for b in range(nb):
+        assert cnt[b] == min(b + 1, 2)
+        assert b in idx[b, : cnt[b]].tolist()
+        assert (idx[b, : cnt[b]] <= b).all()
+
+
+def test_bs_select_all_blocks_closed_form():
+    rng = np.random.default_rng(6)
+    N, d = 64 * 9, 8
+    q, k = rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    idx, cnt = orc.bs_select(q, k, 0.3, 100)
+    for b in range(9):
+        assert cnt[b] == b + 1 and idx[b, : b + 1].tolist() == list(range(b + 1))
+
+
+# ------------------------------------------------------ VS index build
+
+def test_vs_groups_loops():
+    s = [0, 10, 74, 75, 140, 205, 206, 400, 464, 529, 1000]
+    got = orc.vs_groups(np.array(s)).tolist()
+    ref = []
+    a = b = s[0]
+    for o in s[1:]:
+        if o - b <= 64:
+            b = o
+        else:
+            ref.append([a, b])
+            a = b = o
+    ref.append([a, b])
+    assert got == ref
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_vs_index_reproduces_mask(seed):
+    """Index invariants: (groups, per-block verticals) describe exactly the
+    definitional VS mask, and no key appears twice in a block."""
+    rng = np.random.default_rng(seed)
+    N = 64 * 12
+    S = np.unique(np.concatenate([[0], rng.choice(N, 25 + 10 * seed, replace=False)]))
+    V = np.unique(rng.choice(N, 30, replace=False))
+    groups, vcnt, vidx = orc.vs_build_index(V, S, N)
+    ref = orc.mask_vs(np.arange(N), N, V, S)
+    got = np.zeros((N, N), bool)
+    for i in range(N):
+        b = i // 64
+        r0 = 64 * b
+        band = np.zeros(N, bool)
+        for a_g, b_g in groups:
+            lo, hi = max(0, r0 - b_g), r0 + 63 - a_g
+            if hi >= 0:
+                band[lo:hi + 1] = True
+        vert = np.zeros(N, bool)
+        vert[vidx[b, : vcnt[b]]] = True
+        assert not (band & vert).any()            # de-duplicated
+        got[i] = (band | vert) & (np.arange(N) <= i)
+    assert np.array_equal(got, ref)
+
+
+def test_vs_block_verticals_direct_intervals():
+    rng = np.random.default_rng(21)
+    N = 64 * 10
+    S = np.unique(np.concatenate([[0], rng.choice(N, 30, replace=False)]))
+    V = np.unique(rng.choice(N, 40, replace=False))
+    groups = orc.vs_groups(S)
+    vcnt, vidx = orc.vs_block_verticals(V, groups, N)
+    for b in range(N // 64):
+        r0 = 64 * b
+        ref = [j for j in V if j <= r0 + 63 and
+               not any(r0 - bg <= j <= r0 + 63 - ag for ag, bg in groups)]
+        assert vidx[b, : vcnt[b]].tolist() == ref
