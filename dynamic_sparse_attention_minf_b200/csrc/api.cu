@@ -1,0 +1,385 @@
+// Host side of the libminf C ABI: argument validation, workspace carving,
+// TMA descriptor set-up and kernel dispatch.  See include/minf.h for the
+// contract of every entry point.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "minf_device.cuh"
+#include "minf_internal.h"
+
+using namespace minf;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+
+bool shape_ok(const minf_shape* s) {
+  if (!s) return false;
+  if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->N < 128) return false;
+  if (s->Hq % s->Hkv != 0) return false;
+  if (s->N % 128 != 0) return false;
+  if ((long long)s->B * s->Hq * s->N >= (1ll << 31)) return false;
+  return true;
+}
+
+minf_status check_shape(const minf_shape* s) {
+  if (!shape_ok(s)) return MINF_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return MINF_ERR_UNSUPPORTED;
+  return MINF_OK;
+}
+
+float eff_scale(const minf_shape* s) { return s->scale > 0.f ? s->scale : 1.0f / std::sqrt((float)s->d); }
+
+// Carves consecutive 256-byte-aligned buffers out of a workspace.
+struct Carver {
+  char* base;
+  size_t off;
+  template <class T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off = align_up(off + count * sizeof(T));
+    return p;
+  }
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 2-D bf16 view [rows, d] with a box of 64 columns x box_rows rows, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, long long rows, int d, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+minf_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MINF_OK : MINF_ERR_CUDA; }
+
+// ----------------------------------------------------------- workspace plans
+struct VsEstWs {
+  DevStatus* status;
+  float *part_ml, *row_ml, *v_score, *s_score, *dpart;
+};
+size_t plan_vs_est(const minf_shape* s, int nh, char* ws, VsEstWs* out) {
+  Carver c{ws, 0};
+  const size_t bh = (size_t)s->B * nh;
+  const size_t ntiles = (s->N + 127) / 128;
+  VsEstWs w;
+  w.status = c.take<DevStatus>(kStatusBytes / sizeof(DevStatus));
+  w.part_ml = c.take<float>(bh * ntiles * 64 * 2);
+  w.row_ml = c.take<float>(bh * 64 * 2);
+  w.v_score = c.take<float>(bh * s->N);
+  w.s_score = c.take<float>(bh * s->N);
+  w.dpart = c.take<float>(bh * ntiles * 192);
+  if (out) *out = w;
+  return c.off;
+}
+
+struct BsEstWs {
+  DevStatus* status;
+  float *qbar, *kbar, *scores;
+};
+size_t plan_bs_est(const minf_shape* s, int nh, char* ws, BsEstWs* out) {
+  Carver c{ws, 0};
+  const size_t bh = (size_t)s->B * nh;
+  const size_t nb = s->N / 64;
+  BsEstWs w;
+  w.status = c.take<DevStatus>(kStatusBytes / sizeof(DevStatus));
+  w.qbar = c.take<float>(bh * nb * s->d);
+  w.kbar = c.take<float>(bh * nb * s->d);
+  w.scores = c.take<float>(bh * nb * nb);
+  if (out) *out = w;
+  return c.off;
+}
+
+minf_status attn_common(int pol, const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
+                        const int32_t* heads, int nh, minf_bf16* O, float* lse, void* ws, size_t ws_bytes,
+                        void* stream, AttnParams& p) {
+  minf_status st = check_shape(s);
+  if (st != MINF_OK) return st;
+  if (!Q || !K || !V || !O || !ws) return MINF_ERR_INVALID_ARG;
+  if (nh < 1 || nh > s->Hq || (!heads && pol != POL_DENSE)) return MINF_ERR_INVALID_ARG;
+  if (ws_bytes < kStatusBytes) return MINF_ERR_WORKSPACE_TOO_SMALL;
+  if (((uintptr_t)Q | (uintptr_t)K | (uintptr_t)V | (uintptr_t)O) & 15) return MINF_ERR_INVALID_ARG;
+  p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  p.K = reinterpret_cast<const __nv_bfloat16*>(K);
+  p.V = reinterpret_cast<const __nv_bfloat16*>(V);
+  p.O = reinterpret_cast<__nv_bfloat16*>(O);
+  p.lse = lse;
+  p.heads = heads;
+  p.nh = heads ? nh : s->Hq;
+  p.B = s->B;
+  p.Hq = s->Hq;
+  p.Hkv = s->Hkv;
+  p.N = s->N;
+  p.group = s->Hq / s->Hkv;
+  p.scale_log2 = eff_scale(s) * 1.4426950408889634f;
+  p.status = reinterpret_cast<DevStatus*>(ws);
+  return MINF_OK;
+}
+
+minf_status attn_launch(int pol, const minf_shape* s, const AttnParams& p, void* stream) {
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, p.Q, (long long)s->B * s->Hq * s->N, s->d, 128) ||
+      !make_map(&tk, p.K, (long long)s->B * s->Hkv * s->N, s->d, 64) ||
+      !make_map(&tv, p.V, (long long)s->B * s->Hkv * s->N, s->d, 64))
+    return MINF_ERR_CUDA;
+  return cuda_status(attn_dispatch(s->d, pol, tq, tk, tv, p, (cudaStream_t)stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t minf_vs_wmap_words(int N) { return N > 0 ? (size_t)(N + 64) / 32 + 2 : 0; }
+
+size_t minf_workspace_size(int op, const minf_shape* s, int nh, int k_v, int k_s, int k_b) {
+  (void)k_v;
+  (void)k_s;
+  (void)k_b;
+  if (!shape_ok(s) || nh < 1) return 0;
+  switch (op) {
+    case MINF_OP_ESTIMATE_VS:
+      return plan_vs_est(s, nh, nullptr, nullptr);
+    case MINF_OP_ESTIMATE_BS:
+      return plan_bs_est(s, nh, nullptr, nullptr);
+    case MINF_OP_BUILD_INDEX:
+    case MINF_OP_SPARSE_ATTN_VS:
+    case MINF_OP_SPARSE_ATTN_BS:
+    case MINF_OP_ATTN_ASHAPE:
+    case MINF_OP_DENSE_ATTN:
+      return kStatusBytes;
+    default:
+      return 0;
+  }
+}
+
+minf_status minf_estimate_vs(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const int32_t* heads,
+                             int nh, int last_q, int k_v, int k_s, int32_t* v_idx, int32_t* s_idx, float* v_score,
+                             float* s_score, void* ws, size_t ws_bytes, void* stream) {
+  minf_status st = check_shape(s);
+  if (st != MINF_OK) return st;
+  if (!Q || !K || !heads || !v_idx || !s_idx || !ws) return MINF_ERR_INVALID_ARG;
+  if (nh < 1 || nh > s->Hq || last_q < 1 || last_q > 64) return MINF_ERR_INVALID_ARG;
+  if (k_v < 1 || k_s < 1 || k_v > s->N || k_s > s->N) return MINF_ERR_INVALID_ARG;
+  if (ws_bytes < plan_vs_est(s, nh, nullptr, nullptr)) return MINF_ERR_WORKSPACE_TOO_SMALL;
+  VsEstWs w;
+  plan_vs_est(s, nh, (char*)ws, &w);
+  VsEstParams p;
+  p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  p.K = reinterpret_cast<const __nv_bfloat16*>(K);
+  p.heads = heads;
+  p.nh = nh;
+  p.B = s->B;
+  p.Hq = s->Hq;
+  p.Hkv = s->Hkv;
+  p.N = s->N;
+  p.d = s->d;
+  p.group = s->Hq / s->Hkv;
+  p.last_q = last_q;
+  p.scale_log2 = eff_scale(s) * 1.4426950408889634f;
+  p.part_ml = w.part_ml;
+  p.row_ml = w.row_ml;
+  p.v_score = v_score ? v_score : w.v_score;
+  p.s_score = s_score ? s_score : w.s_score;
+  p.dpart = w.dpart;
+  p.status = w.status;
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = vs_estimate_launch(p, cs);
+  if (e != cudaSuccess) return MINF_ERR_CUDA;
+  TopkRows t;
+  t.scores = p.v_score;
+  t.row_stride = s->N;
+  t.rows = s->B * nh;
+  t.len_mode = 0;
+  t.len = s->N;
+  t.rows_per_group = 1;
+  t.forced_mode = 0;
+  t.k = k_v;
+  t.out_idx = v_idx;
+  t.out_cnt = nullptr;
+  t.status = w.status;
+  e = topk_rows_launch(t, cs);
+  if (e != cudaSuccess) return MINF_ERR_CUDA;
+  t.scores = p.s_score;
+  t.forced_mode = 1;
+  t.k = k_s;
+  t.out_idx = s_idx;
+  return cuda_status(topk_rows_launch(t, cs));
+}
+
+minf_status minf_estimate_bs(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const int32_t* heads,
+                             int nh, int block, int k_b, int32_t* blk_idx, int32_t* blk_cnt, float* blk_score,
+                             void* ws, size_t ws_bytes, void* stream) {
+  minf_status st = check_shape(s);
+  if (st != MINF_OK) return st;
+  if (!Q || !K || !heads || !blk_idx || !blk_cnt || !ws) return MINF_ERR_INVALID_ARG;
+  if (nh < 1 || nh > s->Hq || k_b < 1) return MINF_ERR_INVALID_ARG;
+  if (block != 64) return MINF_ERR_UNSUPPORTED;
+  if (ws_bytes < plan_bs_est(s, nh, nullptr, nullptr)) return MINF_ERR_WORKSPACE_TOO_SMALL;
+  BsEstWs w;
+  plan_bs_est(s, nh, (char*)ws, &w);
+  BsEstParams p;
+  p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  p.K = reinterpret_cast<const __nv_bfloat16*>(K);
+  p.heads = heads;
+  p.nh = nh;
+  p.B = s->B;
+  p.Hq = s->Hq;
+  p.Hkv = s->Hkv;
+  p.N = s->N;
+  p.d = s->d;
+  p.group = s->Hq / s->Hkv;
+  p.scale = eff_scale(s);
+  p.qbar = w.qbar;
+  p.kbar = w.kbar;
+  p.scores = blk_score ? blk_score : w.scores;
+  p.status = w.status;
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = bs_pool_score_launch(p, cs);
+  if (e != cudaSuccess) return MINF_ERR_CUDA;
+  const int nb = s->N / 64;
+  TopkRows t;
+  t.scores = p.scores;
+  t.row_stride = nb;
+  t.rows = s->B * nh * nb;
+  t.len_mode = 1;
+  t.len = nb;
+  t.rows_per_group = nb;
+  t.forced_mode = 2;
+  t.k = k_b;
+  t.out_idx = blk_idx;
+  t.out_cnt = blk_cnt;
+  t.status = w.status;
+  return cuda_status(topk_rows_launch(t, cs));
+}
+
+minf_status minf_build_index(const minf_shape* s, int nh, const int32_t* v_idx, int k_v, const int32_t* s_idx,
+                             int k_s, const minf_vs_index* idx, void* ws, size_t ws_bytes, void* stream) {
+  minf_status st = check_shape(s);
+  if (st != MINF_OK) return st;
+  if (!v_idx || !s_idx || !idx || !ws || nh < 1) return MINF_ERR_INVALID_ARG;
+  if (!idx->grp || !idx->grp_cnt || !idx->tgrp || !idx->tgrp_cnt || !idx->wmap || !idx->vcnt || !idx->vidx)
+    return MINF_ERR_INVALID_ARG;
+  if (k_v < 1 || k_s < 1 || k_v > s->N || k_s > s->N) return MINF_ERR_INVALID_ARG;
+  if (ws_bytes < kStatusBytes) return MINF_ERR_WORKSPACE_TOO_SMALL;
+  VsIndexParams p;
+  p.v_idx = v_idx;
+  p.s_idx = s_idx;
+  p.nh = nh;
+  p.B = s->B;
+  p.N = s->N;
+  p.k_v = k_v;
+  p.k_s = k_s;
+  p.wmap_words = (int)minf_vs_wmap_words(s->N);
+  p.idx = *idx;
+  p.status = reinterpret_cast<DevStatus*>(ws);
+  return cuda_status(vs_index_launch(p, (cudaStream_t)stream));
+}
+
+minf_status minf_sparse_attn_vs(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
+                                const int32_t* heads, int nh, const minf_vs_index* idx, int k_v, int k_s,
+                                minf_bf16* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  minf_status st = attn_common(POL_VS, s, Q, K, V, heads, nh, O, lse, ws, ws_bytes, stream, p);
+  if (st != MINF_OK) return st;
+  if (!idx || !idx->tgrp || !idx->tgrp_cnt || !idx->wmap || !idx->vcnt || !idx->vidx) return MINF_ERR_INVALID_ARG;
+  if (k_v < 1 || k_s < 1 || k_v > s->N || k_s > s->N) return MINF_ERR_INVALID_ARG;
+  p.tgrp = idx->tgrp;
+  p.tgrp_cnt = idx->tgrp_cnt;
+  p.wmap = idx->wmap;
+  p.vcnt = idx->vcnt;
+  p.vidx = idx->vidx;
+  p.k_s = k_s;
+  p.k_v = k_v;
+  p.wmap_words = (int)minf_vs_wmap_words(s->N);
+  return attn_launch(POL_VS, s, p, stream);
+}
+
+minf_status minf_sparse_attn_bs(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
+                                const int32_t* heads, int nh, const int32_t* blk_idx, const int32_t* blk_cnt,
+                                int k_b, minf_bf16* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  minf_status st = attn_common(POL_BS, s, Q, K, V, heads, nh, O, lse, ws, ws_bytes, stream, p);
+  if (st != MINF_OK) return st;
+  if (!blk_idx || !blk_cnt || k_b < 1) return MINF_ERR_INVALID_ARG;
+  p.blk_idx = blk_idx;
+  p.blk_cnt = blk_cnt;
+  p.k_b = k_b;
+  return attn_launch(POL_BS, s, p, stream);
+}
+
+minf_status minf_attn_ashape(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
+                             const int32_t* heads, int nh, int n_sink, int n_local, minf_bf16* O, float* lse,
+                             void* ws, size_t ws_bytes, void* stream) {
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  minf_status st = attn_common(POL_ASHAPE, s, Q, K, V, heads, nh, O, lse, ws, ws_bytes, stream, p);
+  if (st != MINF_OK) return st;
+  if (n_sink < 0 || n_local < 1) return MINF_ERR_INVALID_ARG;
+  p.n_sink = n_sink;
+  p.n_local = n_local;
+  return attn_launch(POL_ASHAPE, s, p, stream);
+}
+
+minf_status minf_dense_attn(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
+                            const int32_t* heads, int nh, minf_bf16* O, float* lse, void* ws, size_t ws_bytes,
+                            void* stream) {
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!heads && s && nh != s->Hq) nh = s->Hq;
+  minf_status st = attn_common(POL_DENSE, s, Q, K, V, heads, nh, O, lse, ws, ws_bytes, stream, p);
+  if (st != MINF_OK) return st;
+  return attn_launch(POL_DENSE, s, p, stream);
+}
+
+minf_status minf_get_device_status(void* ws, void* stream) {
+  if (!ws) return MINF_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MINF_ERR_CUDA;
+  DevStatus h{0, 0};
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return MINF_ERR_CUDA;
+  if (h.code != 0 && cudaMemset(ws, 0, sizeof(h)) != cudaSuccess) return MINF_ERR_CUDA;
+  if (h.code == 0) return MINF_OK;
+  return (minf_status)h.code;
+}
+
+const char* minf_status_string(minf_status s) {
+  switch (s) {
+    case MINF_OK: return "ok";
+    case MINF_ERR_INVALID_ARG: return "invalid argument";
+    case MINF_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MINF_ERR_CUDA: return "CUDA error";
+    case MINF_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MINF_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case MINF_ERR_DEVICE_BOUNDS: return "device index out of range";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

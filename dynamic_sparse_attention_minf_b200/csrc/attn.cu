@@ -1,0 +1,801 @@
+// Causal (sparse) attention mainloop for sm_100a: one CTA per (batch, head,
+// 128-row query tile), warp-specialized.
+//
+//   warps 0-3  softmax warpgroup 0: key tiles 0, 2, 4, ...   (thread = query row)
+//   warps 4-7  softmax warpgroup 1: key tiles 1, 3, 5, ...
+//   warp  8    tcgen05 issuer (one lane) and TMEM owner
+//   warp  9    producer: enumerates the key tiles of the query tile for the
+//              head's pattern, writes each tile's descriptor (column ids and
+//              per-64-row-half membership masks) and stages K/V into shared
+//              memory by TMA (contiguous 64-key chunks) or cp.async (gathered
+//              columns).
+//
+// Per key tile t (128 keys) the issuer computes S = Q K^T into the TMEM
+// buffer of warpgroup t&1; that warpgroup masks and exponentiates S, writes
+// P (bf16) back over S in TMEM and the issuer accumulates O_{t&1} += P V with
+// P read from TMEM.  The two warpgroups keep separate running max / sum and
+// separate O accumulators, merged in the epilogue, so that one warpgroup's
+// exponentials overlap the other's matrix products.
+//
+// The four key sources ("MInference 1.0" summary, "Summary": A-shape,
+// Vertical-Slash, Block-Sparse; and dense causal attention as the baseline):
+//   dense   : keys [0, R+128) in 128-key tiles, causal mask on the last
+//   A-shape : [0, n_sink) and the local band [R - n_local + 1, R + 128),
+//             per element j < n_sink or i - j < n_local
+//   VS      : the union over slash groups of the bands swept by the tile's
+//             rows, then the verticals of both 64-row halves, gathered
+//   BS      : the selected 64-key blocks of both halves, two per tile
+#include "minf_device.cuh"
+#include "minf_internal.h"
+
+namespace minf {
+
+enum { KIND_END = 0, KIND_RANGE = 1, KIND_GATHER = 2 };
+enum { F_MASK = 1, F_CAUSAL = 2, F_ASHAPE = 4 };
+
+struct TileDesc {
+  int kind;
+  int flags;
+  int j0[2];             // RANGE: first key of the two 64-key chunks
+  uint32_t mask[2][4];   // per 64-row half: key-column membership bits
+  int cols[128];         // GATHER: key id of every column
+};
+
+template <int D>
+struct AttnCfg {
+  static constexpr int kThreads = 320;
+  static constexpr int kRegion = 128 * 128;                 // bytes: 128 rows x 128 B
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kKVBytes = 128 * D * 2;
+  static constexpr int kStages = (D == 128) ? 3 : 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + kStages * kKVBytes;
+  static constexpr int kOffDesc = kOffV + kStages * kKVBytes;
+  static constexpr int kOffSCols = kOffDesc + kStages * (int)sizeof(TileDesc);
+  static constexpr int kOffSBits = kOffSCols + 160 * 4;
+  static constexpr int kOffBars = kOffSBits + 160;
+  // barriers: k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], q_full, mma_done
+  static constexpr int kNumBars = 3 * kStages + 8;
+  static constexpr int kOffMisc = kOffBars + kNumBars * 8;
+  static constexpr int kSmem = kOffMisc + 16;
+  static_assert(kSmem <= 232448, "shared memory budget");
+  static constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);
+  static constexpr uint32_t kIdescPV = idesc_bf16(128, D, 0, 1);
+  static constexpr int kColO0 = 256;
+  static constexpr int kColO1 = 256 + D;
+};
+
+__device__ __forceinline__ uint32_t count_mask(int cnt, int wd) {
+  int n = cnt - 32 * wd;
+  if (n >= 32) return 0xFFFFFFFFu;
+  if (n <= 0) return 0u;
+  return (1u << n) - 1u;
+}
+
+// 32 bits of the slash-band bitmap starting at bit position p (bits below 0
+// read as zero).
+__device__ __forceinline__ uint32_t wmap_window(const uint32_t* W, int p) {
+  if (p <= -32) return 0u;
+  if (p < 0) return __ldg(W) << (-p);
+  const int wi = p >> 5;
+  return __funnelshift_r(__ldg(W + wi), __ldg(W + wi + 1), p & 31);
+}
+__device__ __forceinline__ uint32_t wmap_bit(const uint32_t* W, int x) {
+  return (__ldg(W + (x >> 5)) >> (x & 31)) & 1u;
+}
+
+// A wait whose outcome is the same for every lane of the warp (the TMEM
+// accesses that follow are warp-collective).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, DevStatus* st,
+                                          int where) {
+  const bool ok = mbar_wait(bar, parity, abort, st, where);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+template <int D>
+struct Producer {
+  using C = AttnCfg<D>;
+  uint8_t* smem;
+  TileDesc* desc;
+  int* scols;
+  uint8_t* sbits;
+  uint64_t* k_full;
+  uint64_t* v_full;
+  uint64_t* kv_empty;
+  const CUtensorMap* tmK;
+  const CUtensorMap* tmV;
+  const __nv_bfloat16* Kh;  // this (batch, kv head)'s K rows
+  const __nv_bfloat16* Vh;
+  int kv_row0;
+  int R;
+  int N;
+  int lane;
+  int t;
+  int pending;  // stage whose gathered copies are issued but not yet signalled
+  int issued[C::kStages];
+  volatile int* abort;
+  DevStatus* st;
+  bool ok;
+
+  __device__ void flush_pending() {
+    if (pending >= 0) {
+      cp_async_wait<0>();
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&k_full[pending]);
+        mbar_arrive(&v_full[pending]);
+      }
+      pending = -1;
+    }
+  }
+
+  // Claims the stage of tile t; false on abort.
+  __device__ bool acquire(int& stage) {
+    stage = t % C::kStages;
+    if (t >= C::kStages) {
+      flush_pending();
+      if (!warp_wait(&kv_empty[stage], ((t / C::kStages) - 1) & 1, abort, st, 1)) {
+        ok = false;
+        return false;
+      }
+    }
+    return true;
+  }
+
+  // A tile of two 64-key chunks at keys j0a, j0b with per-half mask words
+  // (lane l < 8 holds word (l >> 2, l & 3)).
+  __device__ void emit_range(int j0a, int j0b, uint32_t word, int flags) {
+    if (!ok) return;
+    int stage;
+    if (!acquire(stage)) return;
+    TileDesc& dd = desc[stage];
+    const bool full = __all_sync(0xFFFFFFFFu, lane >= 8 || word == 0xFFFFFFFFu);
+    if (lane < 8) dd.mask[lane >> 2][lane & 3] = word;
+    if (lane == 0) {
+      dd.kind = KIND_RANGE;
+      dd.flags = flags | (full ? 0 : F_MASK);
+      dd.j0[0] = j0a;
+      dd.j0[1] = j0b;
+    }
+    __threadfence_block();
+    __syncwarp();
+    if (lane == 0) {
+      issued[stage] = t;
+      uint8_t* kb = smem + C::kOffK + stage * C::kKVBytes;
+      uint8_t* vb = smem + C::kOffV + stage * C::kKVBytes;
+      mbar_arrive_expect_tx(&k_full[stage], C::kKVBytes);
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) {
+        tma_load_2d(kb + h * C::kRegion, tmK, &k_full[stage], 64 * h, kv_row0 + j0a);
+        tma_load_2d(kb + h * C::kRegion + 8192, tmK, &k_full[stage], 64 * h, kv_row0 + j0b);
+      }
+      mbar_arrive_expect_tx(&v_full[stage], C::kKVBytes);
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) {
+        tma_load_2d(vb + h * C::kRegion, tmV, &v_full[stage], 64 * h, kv_row0 + j0a);
+        tma_load_2d(vb + h * C::kRegion + 8192, tmV, &v_full[stage], 64 * h, kv_row0 + j0b);
+      }
+    }
+    ++t;
+  }
+
+  // A gathered tile of the first cnt staged columns (1 <= cnt <= 128).
+  __device__ void emit_gather(int cnt) {
+    if (!ok) return;
+    int stage;
+    if (!acquire(stage)) return;
+    TileDesc& dd = desc[stage];
+    int any_late = 0;
+#pragma unroll
+    for (int wd = 0; wd < 4; ++wd) {
+      const int c = 32 * wd + lane;
+      const int j = (c < cnt) ? scols[c] : scols[0];
+      dd.cols[c] = j;
+      any_late |= (c < cnt && j > R);
+      const uint32_t b = (c < cnt) ? sbits[c] : 0u;
+      const uint32_t w0 = __ballot_sync(0xFFFFFFFFu, b & 1u);
+      const uint32_t w1 = __ballot_sync(0xFFFFFFFFu, b & 2u);
+      if (lane == 0) {
+        dd.mask[0][wd] = w0;
+        dd.mask[1][wd] = w1;
+      }
+    }
+    any_late = __any_sync(0xFFFFFFFFu, any_late);
+    if (lane == 0) {
+      dd.kind = KIND_GATHER;
+      dd.flags = F_MASK | (any_late ? F_CAUSAL : 0);
+    }
+    __threadfence_block();
+    __syncwarp();
+    // cp.async gather of 128 K and V rows into the 128B-swizzled layout.
+    constexpr int CH = D * 2 / 16;  // 16-byte chunks per row
+    const uint32_t kb = smem_u32(smem + C::kOffK + stage * C::kKVBytes);
+    const uint32_t vb = smem_u32(smem + C::kOffV + stage * C::kKVBytes);
+#pragma unroll 4
+    for (int it = 0; it < 128 * CH / 32; ++it) {
+      const int idx = it * 32 + lane;
+      const int c = idx / CH;
+      const int q = idx % CH;
+      const int j = dd.cols[c];
+      const uint32_t off = (q >> 3) * C::kRegion + c * 128 + (((q & 7) ^ (c & 7)) << 4);
+      cp_async16(kb + off, Kh + (size_t)j * D + q * 8);
+      cp_async16(vb + off, Vh + (size_t)j * D + q * 8);
+    }
+    cp_async_commit();
+    if (lane == 0) issued[stage] = t;
+    // signal the previous gathered tile, keep this one in flight
+    if (pending >= 0) {
+      cp_async_wait<1>();
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&k_full[pending]);
+        mbar_arrive(&v_full[pending]);
+      }
+    }
+    pending = stage;
+    ++t;
+  }
+
+  __device__ void emit_end() {
+    flush_pending();
+    for (int e = 0; e < 2 && ok; ++e) {
+      int stage;
+      if (!acquire(stage)) return;
+      if (lane == 0) {
+        desc[stage].kind = KIND_END;
+        issued[stage] = -1;
+        mbar_arrive(&k_full[stage]);
+      }
+      __syncwarp();
+      ++t;
+    }
+  }
+
+  // Appends a warp-wide batch of candidate columns to the staging list,
+  // emitting gathered tiles whenever 128 are ready.  n_staged is warp-uniform.
+  __device__ void append(bool keep, int j, uint32_t bits, int& n_staged) {
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+    const int pos = n_staged + __popc(bal & ((1u << lane) - 1u));
+    if (keep) {
+      scols[pos] = j;
+      sbits[pos] = (uint8_t)bits;
+    }
+    n_staged += __popc(bal);
+    __syncwarp();
+    if (n_staged >= 128) {
+      emit_gather(128);
+      __syncwarp();
+      const int rest = n_staged - 128;
+      int mj = 0;
+      uint8_t mb = 0;
+      if (lane < rest) {
+        mj = scols[128 + lane];
+        mb = sbits[128 + lane];
+      }
+      __syncwarp();
+      if (lane < rest) {
+        scols[lane] = mj;
+        sbits[lane] = mb;
+      }
+      n_staged = rest;
+      __syncwarp();
+    }
+  }
+
+  // Waits (bounded, ignoring the abort flag) until every copy this producer
+  // started has landed, so that the CTA never exits with copies in flight.
+  __device__ void drain() {
+    cp_async_wait<0>();
+    __syncwarp();
+    if (lane == 0) {
+      int dummy = 0;
+      for (int s = 0; s < C::kStages; ++s) {
+        if (issued[s] >= 0) {
+          const uint32_t par = (issued[s] / C::kStages) & 1;
+          mbar_wait(&k_full[s], par, &dummy, st, 9);
+          mbar_wait(&v_full[s], par, &dummy, st, 9);
+        }
+      }
+    }
+    __syncwarp();
+  }
+};
+
+template <int D, int POL>
+__device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi, int qt) {
+  const int R = qt * 128;
+  const int lane = P.lane;
+  if (POL == POL_DENSE) {
+    for (int m = 0; m <= qt && P.ok; ++m) {
+      P.emit_range(128 * m, 128 * m + 64, 0xFFFFFFFFu, m == qt ? F_CAUSAL : 0);
+    }
+  } else if (POL == POL_ASHAPE) {
+    const int lloc = max(0, R - p.n_local + 1);
+    int lo[2], hi_[2], n_iv = 0;
+    if (p.n_sink >= lloc) {
+      lo[0] = 0; hi_[0] = R + 127; n_iv = 1;
+    } else {
+      if (p.n_sink > 0) { lo[n_iv] = 0; hi_[n_iv] = p.n_sink - 1; ++n_iv; }
+      lo[n_iv] = lloc; hi_[n_iv] = R + 127; ++n_iv;
+    }
+    const int far_edge = R + 127 - p.n_local;   // keys <= this may leave some row's window
+    for (int v = 0; v < n_iv; ++v) {
+      for (int j0 = lo[v]; j0 <= hi_[v] && P.ok; j0 += 128) {
+        const int cnt = min(128, hi_[v] - j0 + 1);
+        const uint32_t word = (lane < 8) ? count_mask(cnt, lane & 3) : 0xFFFFFFFFu;
+        int flags = (j0 + cnt - 1 > R) ? F_CAUSAL : 0;
+        if (max(j0, p.n_sink) <= min(j0 + cnt - 1, far_edge)) flags |= F_ASHAPE;
+        P.emit_range(j0, j0 + 64, word, flags);
+      }
+    }
+  } else if (POL == POL_VS) {
+    const size_t hrow = (size_t)b * p.nh + hi;
+    const int* tg = p.tgrp + hrow * p.k_s * 2;
+    const int G = p.tgrp_cnt[hrow];
+    const uint32_t* W = p.wmap + hrow * p.wmap_words;
+    // slash bands: ascending keys = descending offsets
+    for (int g = G - 1; g >= 0 && P.ok; --g) {
+      const int A = tg[2 * g], Bo = tg[2 * g + 1];
+      const int hi_key = min(R + 127 - A, p.N - 1);
+      if (hi_key < 0) continue;
+      const int lo_key = max(0, R - Bo);
+      for (int j0 = lo_key; j0 <= hi_key && P.ok; j0 += 128) {
+        const int cnt = min(128, hi_key - j0 + 1);
+        uint32_t word = 0xFFFFFFFFu;
+        if (lane < 8) {
+          const int hh = lane >> 2, wd = lane & 3;
+          const int x0 = R + 64 * hh - j0 + 63 - 32 * wd;
+          word = __brev(wmap_window(W, x0 - 31)) & count_mask(cnt, wd);
+        }
+        P.emit_range(j0, j0 + 64, word, (j0 + cnt - 1 > R) ? F_CAUSAL : 0);
+      }
+    }
+    // verticals: V_{b1} (both halves as applicable), then V_{b0} on half-1 bands
+    const int nb = p.N / 64;
+    const int b0 = R / 64, b1 = b0 + 1;
+    const int* vl1 = p.vidx + (hrow * nb + b1) * (size_t)p.k_v;
+    const int* vl0 = p.vidx + (hrow * nb + b0) * (size_t)p.k_v;
+    const int c1 = min(p.vcnt[hrow * nb + b1], p.k_v);
+    const int c0 = min(p.vcnt[hrow * nb + b0], p.k_v);
+    int n_staged = 0;
+    for (int base = 0; base < c1 && P.ok; base += 32) {
+      const int idx = base + lane;
+      int j = (idx < c1) ? vl1[idx] : 0;
+      if (j < 0 || j > R + 127) { if (idx < c1) report(P.st, MINF_ERR_DEVICE_BOUNDS, 20); j = 0; }
+      const uint32_t h0 = (idx < c1 && j <= R + 63 && !wmap_bit(W, R - j + 63)) ? 1u : 0u;
+      P.append(idx < c1, j, h0 | 2u, n_staged);
+    }
+    for (int base = 0; base < c0 && P.ok; base += 32) {
+      const int idx = base + lane;
+      int j = (idx < c0) ? vl0[idx] : 0;
+      if (j < 0 || j > R + 63) { if (idx < c0) report(P.st, MINF_ERR_DEVICE_BOUNDS, 21); j = 0; }
+      const bool keep = (idx < c0) && wmap_bit(W, R + 127 - j);
+      P.append(keep, j, 1u, n_staged);
+    }
+    if (n_staged > 0 && P.ok) P.emit_gather(n_staged);
+  } else if (POL == POL_BS) {
+    const size_t hrow = (size_t)b * p.nh + hi;
+    const int nb = p.N / 64;
+    const int b0 = R / 64, b1 = b0 + 1;
+    const int* s0 = p.blk_idx + (hrow * nb + b0) * (size_t)p.k_b;
+    const int* s1 = p.blk_idx + (hrow * nb + b1) * (size_t)p.k_b;
+    const int n0 = min(p.blk_cnt[hrow * nb + b0], p.k_b);
+    const int n1 = min(p.blk_cnt[hrow * nb + b1], p.k_b);
+    int n_staged = 0;
+    // staging of whole key blocks; a tile takes two
+    auto flush_pairs = [&](bool final_) {
+      while (n_staged >= 2 || (final_ && n_staged == 1)) {
+        const int ca = P.scols[0];
+        const uint32_t ba = P.sbits[0];
+        const bool two = n_staged >= 2;
+        const int cb = two ? P.scols[1] : ca;
+        const uint32_t bb = two ? P.sbits[1] : 0u;
+        uint32_t word = 0xFFFFFFFFu;
+        if (lane < 8) {
+          const int hh = lane >> 2, wd = lane & 3;
+          const uint32_t bits = (wd < 2) ? ba : bb;
+          word = ((bits >> hh) & 1u) ? 0xFFFFFFFFu : 0u;
+        }
+        const int flags = (max(ca, cb) >= b0) ? F_CAUSAL : 0;
+        P.emit_range(64 * ca, 64 * cb, word, flags);
+        __syncwarp();
+        const int used = two ? 2 : 1;
+        int mj = 0;
+        uint8_t mb = 0;
+        const int rest = n_staged - used;
+        if (lane < rest) { mj = P.scols[used + lane]; mb = P.sbits[used + lane]; }
+        __syncwarp();
+        if (lane < rest) { P.scols[lane] = mj; P.sbits[lane] = mb; }
+        n_staged = rest;
+        __syncwarp();
+        if (!P.ok) return;
+      }
+    };
+    for (int base = 0; base < n1 && P.ok; base += 32) {
+      const int idx = base + lane;
+      int c = (idx < n1) ? s1[idx] : 0;
+      if (c < 0 || c > b1) { if (idx < n1) report(P.st, MINF_ERR_DEVICE_BOUNDS, 22); c = 0; }
+      // member of half 0's list?  (binary search in s0)
+      int lo = 0, hi2 = n0;
+      while (lo < hi2) { const int mid = (lo + hi2) >> 1; if (s0[mid] < c) lo = mid + 1; else hi2 = mid; }
+      const uint32_t h0 = (lo < n0 && s0[lo] == c) ? 1u : 0u;
+      const bool keep = idx < n1;
+      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+      // append one at a time through the shared staging list in order
+      const int pos = n_staged + __popc(bal & ((1u << lane) - 1u));
+      if (keep) { P.scols[pos] = c; P.sbits[pos] = (uint8_t)(h0 | 2u); }
+      n_staged += __popc(bal);
+      __syncwarp();
+      flush_pairs(false);
+    }
+    for (int base = 0; base < n0 && P.ok; base += 32) {
+      const int idx = base + lane;
+      int c = (idx < n0) ? s0[idx] : 0;
+      if (c < 0 || c > b0) { if (idx < n0) report(P.st, MINF_ERR_DEVICE_BOUNDS, 23); c = 0; }
+      int lo = 0, hi2 = n1;
+      while (lo < hi2) { const int mid = (lo + hi2) >> 1; if (s1[mid] < c) lo = mid + 1; else hi2 = mid; }
+      const bool in1 = (lo < n1 && s1[lo] == c);
+      const bool keep = idx < n0 && !in1;
+      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+      const int pos = n_staged + __popc(bal & ((1u << lane) - 1u));
+      if (keep) { P.scols[pos] = c; P.sbits[pos] = 1u; }
+      n_staged += __popc(bal);
+      __syncwarp();
+      flush_pairs(false);
+    }
+    if (P.ok) flush_pairs(true);
+  }
+}
+
+template <int D, int POL>
+__global__ void __launch_bounds__(320, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = AttnCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int nqt = p.N / 128;
+  const int qt = nqt - 1 - blockIdx.x;  // heaviest query tiles first
+  const int hi = blockIdx.y;
+  const int b = blockIdx.z;
+  const int head = p.heads ? p.heads[hi] : hi;
+  const int kvh = head / p.group;
+  const int R = qt * 128;
+
+  TileDesc* desc = reinterpret_cast<TileDesc*>(smem + C::kOffDesc);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
+  uint64_t* k_full = bars;
+  uint64_t* v_full = bars + C::kStages;
+  uint64_t* kv_empty = bars + 2 * C::kStages;
+  uint64_t* s_full = bars + 3 * C::kStages;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* q_full = o_done + 2;
+  uint64_t* mma_done = q_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  if ((smem_u32(smem) & 1023u) != 0u) {  // the swizzled layouts need 1 KiB alignment
+    if (threadIdx.x == 0) report(p.status, MINF_ERR_DEVICE_BOUNDS, 99);
+    return;
+  }
+  if (head < 0 || head >= p.Hq) {
+    if (threadIdx.x == 0) report(p.status, MINF_ERR_DEVICE_BOUNDS, 98);
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&p_full[w], 128);
+      mbar_init(&o_done[w], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(mma_done, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ producer
+    Producer<D> P;
+    P.smem = smem;
+    P.desc = desc;
+    P.scols = reinterpret_cast<int*>(smem + C::kOffSCols);
+    P.sbits = smem + C::kOffSBits;
+    P.k_full = k_full;
+    P.v_full = v_full;
+    P.kv_empty = kv_empty;
+    P.tmK = &tmK;
+    P.tmV = &tmV;
+    P.kv_row0 = (b * p.Hkv + kvh) * p.N;
+    P.Kh = p.K + (size_t)P.kv_row0 * D;
+    P.Vh = p.V + (size_t)P.kv_row0 * D;
+    P.R = R;
+    P.N = p.N;
+    P.lane = lane;
+    P.t = 0;
+    P.pending = -1;
+    for (int s = 0; s < C::kStages; ++s) P.issued[s] = -1;
+    P.abort = abort;
+    P.st = p.status;
+    P.ok = true;
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_arrive_expect_tx(q_full, C::kQBytes);
+      const int qrow = (b * p.Hq + head) * p.N + R;
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) tma_load_2d(smem + C::kOffQ + h * C::kRegion, &tmQ, q_full, 64 * h, qrow);
+    }
+    __syncwarp();
+    produce_tiles<D, POL>(P, p, b, hi, qt);
+    P.emit_end();
+    P.flush_pending();
+    P.drain();
+    if (lane == 0) {
+      int dummy = 0;
+      mbar_wait(q_full, 0, &dummy, p.status, 8);
+    }
+  } else if (warp == 8) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t qaddr = smem_u32(smem + C::kOffQ);
+      auto issue_pv = [&](int tp) -> bool {
+        const int wp = tp & 1;
+        const int sp = tp % C::kStages;
+        if (!mbar_wait(&p_full[wp], (tp >> 1) & 1, abort, p.status, 3)) return false;
+        if (!mbar_wait(&v_full[sp], (tp / C::kStages) & 1, abort, p.status, 4)) return false;
+        tc_fence_after();
+        const uint32_t vaddr = smem_u32(smem + C::kOffV + sp * C::kKVBytes);
+        const uint32_t d_tmem = tmem + (wp ? C::kColO1 : C::kColO0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, C::kRegion, 1024);
+          umma_ts(d_tmem, tmem + wp * 128 + kk * 8, bd, C::kIdescPV, (tp >= 2 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&o_done[wp]);
+        umma_commit(&kv_empty[sp]);
+        return true;
+      };
+      bool ok = mbar_wait(q_full, 0, abort, p.status, 2);
+      int t = 0, pend = -1;
+      while (ok) {
+        const int st = t % C::kStages;
+        if (!mbar_wait(&k_full[st], (t / C::kStages) & 1, abort, p.status, 5)) { ok = false; break; }
+        if (desc[st].kind == KIND_END) break;
+        tc_fence_after();
+        const int w = t & 1;
+        const uint32_t kaddr = smem_u32(smem + C::kOffK + st * C::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kRegion + (kk & 3) * 32;
+          const uint64_t ad = sdesc_sw128(qaddr + off, 16, 1024);
+          const uint64_t bd = sdesc_sw128(kaddr + off, 16, 1024);
+          umma_ss(tmem + w * 128, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[w]);
+        if (pend >= 0 && !issue_pv(pend)) { ok = false; pend = -1; break; }
+        pend = t;
+        ++t;
+      }
+      if (ok && pend >= 0) issue_pv(pend);
+      umma_commit(mma_done);
+      int dummy = 0;
+      mbar_wait(mma_done, 0, &dummy, p.status, 7);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int wg = warp >> 2;
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const int i = R + r;
+    const int half = r >> 6;
+    const float sl2 = p.scale_log2;
+    const uint32_t srow = tmem + ((uint32_t)(q4 * 32) << 16);
+    float m_run = -INFINITY, l_run = 0.f;
+    int n = 0;
+    for (int t = wg;; t += 2) {
+      const int st = t % C::kStages;
+      if (!warp_wait(&k_full[st], (t / C::kStages) & 1, abort, p.status, 10)) break;
+      const TileDesc& dd = desc[st];
+      const int kind = dd.kind;
+      if (kind == KIND_END) break;
+      if (!warp_wait(&s_full[wg], n & 1, abort, p.status, 11)) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(srow + wg * 128 + c4 * 32, sr[c4]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) reg_fence(sr[c4]);
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+
+      const int flags = dd.flags;
+      if (flags & F_MASK) {
+        const uint32_t mw0 = dd.mask[half][0], mw1 = dd.mask[half][1];
+        const uint32_t mw2 = dd.mask[half][2], mw3 = dd.mask[half][3];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const uint32_t mw = (c < 32) ? mw0 : (c < 64) ? mw1 : (c < 96) ? mw2 : mw3;
+          if (!((mw >> (c & 31)) & 1u)) s[c] = -INFINITY;
+        }
+      }
+      if (flags & (F_CAUSAL | F_ASHAPE)) {
+        const bool causal = flags & F_CAUSAL;
+        const bool ash = flags & F_ASHAPE;
+        if (kind == KIND_RANGE) {
+          const int ja = dd.j0[0], jb = dd.j0[1];
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const int j = ((c < 64) ? ja : jb) + (c & 63);
+            bool drop = causal && (j > i);
+            drop |= ash && (j >= p.n_sink) && (i - j >= p.n_local);
+            if (drop) s[c] = -INFINITY;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const int j = dd.cols[c];
+            if (causal && j > i) s[c] = -INFINITY;
+          }
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      const float m_new = fmaxf(m_run, mx * sl2);
+      float alpha = 1.f;
+      const bool resc = m_new > m_run + 8.f;
+      if (resc) {
+        alpha = fast_exp2(m_run - m_new);
+        m_run = m_new;
+      }
+      const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+      float lsum = 0.f;
+      // lazy correction of the running output (rare after the first tiles)
+      if (__any_sync(0xFFFFFFFFu, resc && n > 0)) {
+        if (!warp_wait(&o_done[wg], (n - 1) & 1, abort, p.status, 12)) break;
+        tc_fence_after();
+        const uint32_t orow = srow + (wg ? C::kColO1 : C::kColO0);
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(orow + c0, o);
+          tmem_wait_ld();
+          reg_fence(o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(orow + c0, o);
+        }
+      }
+      // P = exp2(s * scale * log2 e - m), written as bf16 pairs over S's columns
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = fast_exp2(fmaf(s[c4 * 32 + e], sl2, -msub));
+          const float p1 = fast_exp2(fmaf(s[c4 * 32 + e + 1], sl2, -msub));
+          lsum += p0 + p1;
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(srow + wg * 128 + c4 * 16, pk);
+      }
+      l_run = l_run * alpha + lsum;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[wg]);
+      ++n;
+    }
+    // ----------------------------------------------------------- epilogue
+    bool ok = !*abort;
+    if (ok && n > 0) ok = warp_wait(&o_done[wg], (n - 1) & 1, abort, p.status, 13);
+    named_bar_sync(1, 256);
+    float* xch = reinterpret_cast<float*>(smem + C::kOffK);  // all S MMAs are done: K stage 0 is free
+    xch[(wg * 128 + r) * 4 + 0] = m_run;
+    xch[(wg * 128 + r) * 4 + 1] = l_run;
+    xch[(wg * 128 + r) * 4 + 2] = __int_as_float(n);
+    named_bar_sync(1, 256);
+    const float m0 = xch[r * 4 + 0], l0 = xch[r * 4 + 1];
+    const float m1 = xch[(128 + r) * 4 + 0], l1 = xch[(128 + r) * 4 + 1];
+    const int n0 = __float_as_int(xch[r * 4 + 2]);
+    const int n1 = __float_as_int(xch[(128 + r) * 4 + 2]);
+    ok = ok && !*abort;
+    if (ok) {
+      const float mt = fmaxf(m0, m1);
+      const float a0 = (l0 > 0.f) ? fast_exp2(m0 - mt) : 0.f;
+      const float a1 = (l1 > 0.f) ? fast_exp2(m1 - mt) : 0.f;
+      const float L = l0 * a0 + l1 * a1;
+      const float inv = (L > 0.f) ? 1.f / L : 0.f;
+      const float c0f = a0 * inv, c1f = a1 * inv;
+      tc_fence_after();
+      __nv_bfloat16* orow_g = p.O + ((size_t)(b * p.Hq + head) * p.N + i) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 2; cc += 32) {
+        const int col = wg * (D / 2) + cc;
+        uint32_t x0[32], x1[32];
+        if (n0 > 0) tmem_ld32(srow + C::kColO0 + col, x0);
+        if (n1 > 0) tmem_ld32(srow + C::kColO1 + col, x1);
+        tmem_wait_ld();
+        reg_fence(x0);
+        reg_fence(x1);
+        uint32_t outw[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float v0 = 0.f, v1 = 0.f;
+          if (n0 > 0) { v0 += __uint_as_float(x0[e]) * c0f; v1 += __uint_as_float(x0[e + 1]) * c0f; }
+          if (n1 > 0) { v0 += __uint_as_float(x1[e]) * c1f; v1 += __uint_as_float(x1[e + 1]) * c1f; }
+          outw[e >> 1] = pack_bf16x2(v0, v1);
+        }
+        if (i < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow_g + col);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(outw[4 * v], outw[4 * v + 1], outw[4 * v + 2], outw[4 * v + 3]);
+        }
+      }
+      if (wg == 0 && p.lse != nullptr && i < p.N) {
+        p.lse[(size_t)(b * p.Hq + head) * p.N + i] = (L > 0.f) ? (mt + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ launch
+template <int D, int POL>
+static cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const AttnParams& p, cudaStream_t stream) {
+  using C = AttnCfg<D>;
+  auto kfn = attn_kernel<D, POL>;
+  cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.N / 128, p.nh, p.B);
+  kfn<<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t attn_dispatch(int d, int pol, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const AttnParams& p, cudaStream_t stream) {
+#define MINF_CASE(DD, PP) \
+  if (d == DD && pol == PP) return launch_attn<DD, PP>(tq, tk, tv, p, stream);
+  MINF_CASE(64, POL_DENSE)
+  MINF_CASE(64, POL_ASHAPE)
+  MINF_CASE(64, POL_VS)
+  MINF_CASE(64, POL_BS)
+  MINF_CASE(128, POL_DENSE)
+  MINF_CASE(128, POL_ASHAPE)
+  MINF_CASE(128, POL_VS)
+  MINF_CASE(128, POL_BS)
+#undef MINF_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace minf

@@ -1,0 +1,450 @@
+// Online sparse-index estimation ("MInference 1.0" summary, "Key points",
+// second item):
+//  * Vertical-Slash: the last query rows are scored against all keys; a
+//    softmax over each row gives p_ij, summed per key column (vertical score)
+//    and per diagonal offset i - j (slash score).
+//  * Block-Sparse: queries and keys are mean-pooled over 64-token blocks and
+//    the pooled query of each block is scored against the pooled keys.
+//  * Top-k per score row by radix select, ties to the lower index, output
+//    ascending.
+// All reductions run in a fixed order, so results are bit-reproducible.
+#include "minf_device.cuh"
+#include "minf_internal.h"
+
+namespace minf {
+
+// ===================================================== Vertical-Slash scores
+// One CTA: 64 query rows (the last L <= 64 rows of one head) x 128 keys.
+constexpr int kVsKeys = 128;
+constexpr int kVsDiag = 192;  // diagonals of a 64 x 128 tile (191 used)
+
+template <int D>
+struct VsSmem {
+  float q[D][64];                 // transposed last rows of Q
+  float k[D][kVsKeys + 4];        // transposed key tile
+};
+
+// Scores of the CTA's 64 x 128 tile in the log2 domain: acc[a][b] holds row
+// ty*4+a, column tx*8+b.
+template <int D>
+__device__ __forceinline__ void vs_tile_scores(const VsEstParams& p, VsSmem<D>& sm, int b, int head, int kvh,
+                                               int j0, float (&acc)[4][8]) {
+  const int tid = threadIdx.x;
+  const int L = p.last_q;
+  const __nv_bfloat16* qh = p.Q + ((size_t)(b * p.Hq + head) * p.N + (p.N - L)) * D;
+  const __nv_bfloat16* kh = p.K + ((size_t)(b * p.Hkv + kvh) * p.N + j0) * D;
+  for (int e = tid; e < 64 * D; e += blockDim.x) {
+    const int r = e / D, dd = e % D;
+    sm.q[dd][r] = (r < L) ? __bfloat162float(qh[(size_t)r * D + dd]) : 0.f;
+  }
+  for (int e = tid; e < kVsKeys * D; e += blockDim.x) {
+    const int c = e / D, dd = e % D;
+    sm.k[dd][c] = (j0 + c < p.N) ? __bfloat162float(kh[(size_t)c * D + dd]) : 0.f;
+  }
+  __syncthreads();
+  const int ty = tid >> 4, tx = tid & 15;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
+#pragma unroll 4
+  for (int dd = 0; dd < D; ++dd) {
+    const float4 qv = *reinterpret_cast<const float4*>(&sm.q[dd][ty * 4]);
+    const float4 k0 = *reinterpret_cast<const float4*>(&sm.k[dd][tx * 8]);
+    const float4 k1 = *reinterpret_cast<const float4*>(&sm.k[dd][tx * 8 + 4]);
+    const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
+    const float kb[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(qa[a], kb[c], acc[a][c]);
+  }
+  // scale into log2 units and apply the causal / range mask
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int r = ty * 4 + a;
+    const int i = p.N - L + r;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int j = j0 + tx * 8 + c;
+      const bool ok = (r < L) && (j <= i) && (j < p.N);
+      acc[a][c] = ok ? acc[a][c] * p.scale_log2 : -INFINITY;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) vs_pass1_kernel(const VsEstParams p) {
+  extern __shared__ __align__(16) uint8_t smraw[];
+  VsSmem<D>& sm = *reinterpret_cast<VsSmem<D>*>(smraw);
+  const int tile = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
+  const int head = p.heads[hi];
+  if (head < 0 || head >= p.Hq) {
+    if (threadIdx.x == 0) report(p.status, MINF_ERR_DEVICE_BOUNDS, 30);
+    return;
+  }
+  float acc[4][8];
+  vs_tile_scores<D>(p, sm, b, head, head / p.group, tile * kVsKeys, acc);
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  const int ntiles = gridDim.x;
+  float* out = p.part_ml + (((size_t)(b * p.nh + hi) * ntiles + tile) * 64) * 2;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) m = fmaxf(m, acc[a][c]);
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    float l = 0.f;
+    if (m != -INFINITY) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) l += exp2f(acc[a][c] - m);
+    }
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, o);
+    if (tx == 0) {
+      out[(ty * 4 + a) * 2 + 0] = m;
+      out[(ty * 4 + a) * 2 + 1] = l;
+    }
+  }
+}
+
+// Combines the per-tile (max, sum) of each row in a fixed order.
+__global__ void __launch_bounds__(256) vs_combine_kernel(const VsEstParams p, int ntiles) {
+  const int r = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
+  const float* part = p.part_ml + ((size_t)(b * p.nh + hi) * ntiles) * 64 * 2;
+  __shared__ float red[256];
+  float m = -INFINITY;
+  for (int t = threadIdx.x; t < ntiles; t += 256) m = fmaxf(m, part[((size_t)t * 64 + r) * 2]);
+  red[threadIdx.x] = m;
+  __syncthreads();
+  for (int s = 128; s > 0; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] = fmaxf(red[threadIdx.x], red[threadIdx.x + s]);
+    __syncthreads();
+  }
+  const float M = red[0];
+  __syncthreads();
+  float l = 0.f;
+  if (M != -INFINITY) {
+    for (int t = threadIdx.x; t < ntiles; t += 256) {
+      const float mt = part[((size_t)t * 64 + r) * 2], lt = part[((size_t)t * 64 + r) * 2 + 1];
+      if (mt != -INFINITY) l += lt * exp2f(mt - M);
+    }
+  }
+  red[threadIdx.x] = l;
+  __syncthreads();
+  for (int s = 128; s > 0; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    float* o = p.row_ml + ((size_t)(b * p.nh + hi) * 64 + r) * 2;
+    o[0] = M;
+    o[1] = (red[0] > 0.f) ? 1.f / red[0] : 0.f;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) vs_pass2_kernel(const VsEstParams p) {
+  extern __shared__ __align__(16) uint8_t smraw[];
+  VsSmem<D>& sm = *reinterpret_cast<VsSmem<D>*>(smraw);
+  const int tile = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
+  const int head = p.heads[hi];
+  if (head < 0 || head >= p.Hq) return;
+  const int j0 = tile * kVsKeys;
+  float acc[4][8];
+  vs_tile_scores<D>(p, sm, b, head, head / p.group, j0, acc);
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const float* rml = p.row_ml + (size_t)(b * p.nh + hi) * 64 * 2;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const float m = rml[(ty * 4 + a) * 2], il = rml[(ty * 4 + a) * 2 + 1];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[a][c] = (acc[a][c] == -INFINITY) ? 0.f : exp2f(acc[a][c] - m) * il;
+  }
+  __syncthreads();  // the key tile is no longer needed: reuse shared memory
+  float* P = reinterpret_cast<float*>(smraw);               // [64][129]
+  float* colp = P + 64 * 129;                               // [16][128]
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) P[(ty * 4 + a) * 129 + tx * 8 + c] = acc[a][c];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float cs = 0.f;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) cs += acc[a][c];
+    colp[ty * 128 + tx * 8 + c] = cs;
+  }
+  __syncthreads();
+  const size_t bh = (size_t)(b * p.nh + hi);
+  if (tid < kVsKeys) {
+    float v = 0.f;
+#pragma unroll
+    for (int y = 0; y < 16; ++y) v += colp[y * 128 + tid];
+    if (j0 + tid < p.N) p.v_score[bh * p.N + j0 + tid] = v;
+  }
+  // diagonal k = r - c + 127 of the tile, summed over rows in ascending order
+  if (tid < 191) {
+    const int k = tid;
+    float dsum = 0.f;
+    const int rlo = max(0, k - 127), rhi = min(63, k);
+    for (int r = rlo; r <= rhi; ++r) dsum += P[r * 129 + (r - k + 127)];
+    p.dpart[(bh * gridDim.x + tile) * kVsDiag + k] = dsum;
+  }
+}
+
+// sigma_o = sum of the (at most two) tiles' diagonal partials holding offset o.
+__global__ void __launch_bounds__(256) vs_slash_kernel(const VsEstParams p, int ntiles) {
+  const int o = blockIdx.x * 256 + threadIdx.x;
+  const int hi = blockIdx.y, b = blockIdx.z;
+  if (o >= p.N) return;
+  const size_t bh = (size_t)(b * p.nh + hi);
+  const int L = p.last_q;
+  // tile t holds offset o at k = o - (N - L - 128 t) + 127 in [0, 190]
+  const int base = p.N - L - o;
+  int tlo = base - 127;  // 128 t >= base - 127
+  tlo = (tlo <= 0) ? 0 : (tlo + 127) / 128;
+  const int thi = min(ntiles - 1, (base + 63) >= 0 ? (base + 63) / 128 : -1);
+  float s = 0.f;
+  for (int t = tlo; t <= thi; ++t) {
+    const int k = 128 * t + 127 - base;
+    if (k >= 0 && k <= 190) s += p.dpart[(bh * ntiles + t) * kVsDiag + k];
+  }
+  p.s_score[bh * p.N + o] = s;
+}
+
+cudaError_t vs_estimate_launch(const VsEstParams& p, cudaStream_t stream) {
+  const int ntiles = (p.N + kVsKeys - 1) / kVsKeys;
+  dim3 grid(ntiles, p.nh, p.B);
+  size_t sm = (p.d == 128) ? sizeof(VsSmem<128>) : sizeof(VsSmem<64>);
+  const size_t sm2 = (64 * 129 + 16 * 128) * sizeof(float);
+  if (sm < sm2) sm = sm2;
+  cudaError_t e;
+  if (p.d == 128) {
+    e = cudaFuncSetAttribute(vs_pass1_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(vs_pass2_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    vs_pass1_kernel<128><<<grid, 256, sm, stream>>>(p);
+  } else {
+    e = cudaFuncSetAttribute(vs_pass1_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(vs_pass2_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    vs_pass1_kernel<64><<<grid, 256, sm, stream>>>(p);
+  }
+  vs_combine_kernel<<<dim3(64, p.nh, p.B), 256, 0, stream>>>(p, ntiles);
+  if (p.d == 128)
+    vs_pass2_kernel<128><<<grid, 256, sm, stream>>>(p);
+  else
+    vs_pass2_kernel<64><<<grid, 256, sm, stream>>>(p);
+  vs_slash_kernel<<<dim3((p.N + 255) / 256, p.nh, p.B), 256, 0, stream>>>(p, ntiles);
+  return cudaGetLastError();
+}
+
+// ================================================================ top-k rows
+constexpr int kTopkThreads = 1024;
+constexpr int kTopkItems = 4;
+
+__device__ __forceinline__ uint32_t order_key(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Inclusive block scan of 64-bit values; returns the inclusive prefix and
+// writes the block total.
+__device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long v, unsigned long long* wsum,
+                                                             unsigned long long& total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, v, o);
+    if (lane >= o) v += y;
+  }
+  if (lane == 31) wsum[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    unsigned long long s = (lane < (int)(blockDim.x >> 5)) ? wsum[lane] : 0ull;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, s, o);
+      if (lane >= o) s += y;
+    }
+    wsum[lane] = s;  // inclusive warp-total prefix
+  }
+  __syncthreads();
+  const unsigned long long before = (w > 0) ? wsum[w - 1] : 0ull;
+  total = wsum[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return v + before;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkRows t) {
+  const int row = blockIdx.x;
+  const int len = (t.len_mode == 0) ? t.len : (row % t.rows_per_group) + 1;
+  const int forced = (t.forced_mode == 0) ? -1 : (t.forced_mode == 1) ? 0 : (row % t.rows_per_group);
+  const float* sc = t.scores + (long long)row * t.row_stride;
+  const int k = min(t.k, len);
+  __shared__ unsigned hist[256];
+  __shared__ unsigned long long wsum[32];
+  __shared__ uint32_t sh_sel, sh_rem;
+  auto key_of = [&](int j) -> uint32_t { return (j == forced) ? 0xFFFFFFFFu : order_key(sc[j]); };
+
+  // radix select of the k-th largest key, 8 bits at a time from the top
+  uint32_t prefix = 0, pmask = 0, rem = (uint32_t)k;
+  for (int shift = 24; shift >= 0 && k > 0; shift -= 8) {
+    for (int x = threadIdx.x; x < 256; x += blockDim.x) hist[x] = 0;
+    __syncthreads();
+    for (int base = 0; base < len; base += blockDim.x) {
+      const int j = base + threadIdx.x;
+      uint32_t digit = 256;
+      if (j < len) {
+        const uint32_t key = key_of(j);
+        if ((key & pmask) == prefix) digit = (key >> shift) & 255u;
+      }
+      const unsigned same = __match_any_sync(0xFFFFFFFFu, digit);
+      if (digit < 256 && (threadIdx.x & 31) == (__ffs(same) - 1)) atomicAdd(&hist[digit], __popc(same));
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t cum = 0, sel = 0;
+      for (int dgt = 255; dgt >= 0; --dgt) {
+        if (cum + hist[dgt] >= rem) {
+          sel = (uint32_t)dgt;
+          break;
+        }
+        cum += hist[dgt];
+      }
+      sh_sel = sel;
+      sh_rem = rem - cum;
+    }
+    __syncthreads();
+    prefix |= sh_sel << shift;
+    pmask |= 255u << shift;
+    rem = sh_rem;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;
+  const unsigned long long need = rem;  // how many keys equal to T are taken (lowest indices)
+  int32_t* out = t.out_idx + (long long)row * t.k;
+  // ordered compaction: element j is taken when key > T, or key == T and
+  // fewer than `need` equal keys precede it
+  unsigned long long gt_before = 0, eq_before = 0;
+  const int chunk = blockDim.x * kTopkItems;
+  for (int base = 0; base < len && k > 0; base += chunk) {
+    uint32_t keys[kTopkItems];
+    unsigned cgt = 0, ceq = 0;
+#pragma unroll
+    for (int e = 0; e < kTopkItems; ++e) {
+      const int j = base + threadIdx.x * kTopkItems + e;
+      keys[e] = (j < len) ? key_of(j) : 0u;
+      const bool valid = j < len;
+      cgt += (valid && keys[e] > T);
+      ceq += (valid && keys[e] == T);
+    }
+    unsigned long long tot;
+    const unsigned long long inc = block_scan_u64(((unsigned long long)cgt << 32) | ceq, wsum, tot);
+    const unsigned long long exc = inc - (((unsigned long long)cgt << 32) | ceq);
+    unsigned long long g = gt_before + (exc >> 32), q = eq_before + (exc & 0xFFFFFFFFull);
+#pragma unroll
+    for (int e = 0; e < kTopkItems; ++e) {
+      const int j = base + threadIdx.x * kTopkItems + e;
+      if (j < len) {
+        if (keys[e] > T) {
+          out[g + min(q, need)] = j;
+          ++g;
+        } else if (keys[e] == T) {
+          if (q < need) out[g + q] = j;
+          ++q;
+        }
+      }
+    }
+    gt_before += tot >> 32;
+    eq_before += tot & 0xFFFFFFFFull;
+  }
+  for (int x = k + threadIdx.x; x < t.k; x += blockDim.x) out[x] = -1;
+  if (t.out_cnt && threadIdx.x == 0) t.out_cnt[row] = k;
+}
+
+cudaError_t topk_rows_launch(const TopkRows& t, cudaStream_t stream) {
+  if (t.rows <= 0) return cudaSuccess;
+  topk_rows_kernel<<<t.rows, kTopkThreads, 0, stream>>>(t);
+  return cudaGetLastError();
+}
+
+// ====================================================== Block-Sparse scores
+// Mean of every 64-row block of Q (listed heads) and K (their KV heads), fp32.
+__global__ void bs_pool_kernel(const BsEstParams p) {
+  const int qb = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
+  const int head = p.heads[hi];
+  if (head < 0 || head >= p.Hq) {
+    if (threadIdx.x == 0) report(p.status, MINF_ERR_DEVICE_BOUNDS, 40);
+    return;
+  }
+  const int nb = p.N / 64;
+  const int kvh = head / p.group;
+  const int dd = threadIdx.x % p.d;
+  const bool isk = threadIdx.x >= p.d;
+  const __nv_bfloat16* src = isk ? p.K + ((size_t)(b * p.Hkv + kvh) * p.N + qb * 64) * p.d
+                                 : p.Q + ((size_t)(b * p.Hq + head) * p.N + qb * 64) * p.d;
+  float s = 0.f;
+  for (int r = 0; r < 64; ++r) s += __bfloat162float(src[(size_t)r * p.d + dd]);
+  float* dst = (isk ? p.kbar : p.qbar) + (((size_t)(b * p.nh + hi) * nb) + qb) * p.d;
+  dst[dd] = s * (1.0f / 64.0f);
+}
+
+// t[b, c] = scale * qbar_b . kbar_c over 64 x 64 tiles with c-tile <= b-tile.
+__global__ void __launch_bounds__(256) bs_score_kernel(const BsEstParams p) {
+  const int ct = blockIdx.x, bt = blockIdx.y, bhz = blockIdx.z;
+  if (ct > bt) return;
+  const int nb = p.N / 64;
+  const float* qb = p.qbar + (size_t)bhz * nb * p.d;
+  const float* kb = p.kbar + (size_t)bhz * nb * p.d;
+  __shared__ float As[32][64 + 4];
+  __shared__ float Bs[32][64 + 4];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < p.d; k0 += 32) {
+    for (int e = tid; e < 64 * 32; e += 256) {
+      const int r = e / 32, kk = e % 32;
+      const int gr = bt * 64 + r, gc = ct * 64 + r;
+      As[kk][r] = (gr < nb) ? qb[(size_t)gr * p.d + k0 + kk] : 0.f;
+      Bs[kk][r] = (gc < nb) ? kb[(size_t)gc * p.d + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < 32; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      const float4 bb = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* out = p.scores + (size_t)bhz * nb * nb;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = bt * 64 + ty * 4 + i;
+    if (r >= nb) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = ct * 64 + tx * 4 + j;
+      if (c < nb) out[(size_t)r * nb + c] = acc[i][j] * p.scale;
+    }
+  }
+}
+
+cudaError_t bs_pool_score_launch(const BsEstParams& p, cudaStream_t stream) {
+  const int nb = p.N / 64;
+  bs_pool_kernel<<<dim3(nb, p.nh, p.B), 2 * p.d, 0, stream>>>(p);
+  const int nt = (nb + 63) / 64;
+  bs_score_kernel<<<dim3(nt, nt, p.B * p.nh), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace minf

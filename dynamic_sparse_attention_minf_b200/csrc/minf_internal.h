@@ -1,0 +1,101 @@
+// Internal declarations shared by the host launcher (api.cu) and the kernel
+// translation units of libminf.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/minf.h"
+
+namespace minf {
+
+struct DevStatus;
+
+enum { POL_DENSE = 0, POL_ASHAPE = 1, POL_VS = 2, POL_BS = 3 };
+
+struct AttnParams {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  __nv_bfloat16* O;
+  float* lse;
+  const int32_t* heads;
+  int nh;
+  int B, Hq, Hkv, N, group;
+  float scale_log2;  // softmax scale * log2(e)
+  // A-shape
+  int n_sink, n_local;
+  // Vertical-Slash index
+  const int32_t* tgrp;
+  const int32_t* tgrp_cnt;
+  const uint32_t* wmap;
+  const int32_t* vcnt;
+  const int32_t* vidx;
+  int k_s, k_v, wmap_words;
+  // Block-Sparse index
+  const int32_t* blk_idx;
+  const int32_t* blk_cnt;
+  int k_b;
+  DevStatus* status;
+};
+
+cudaError_t attn_dispatch(int d, int pol, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const AttnParams& p, cudaStream_t stream);
+
+// ---- estimation / index kernels (estimate.cu, index.cu)
+struct VsEstParams {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  const int32_t* heads;
+  int nh, B, Hq, Hkv, N, d, group, last_q;
+  float scale_log2;
+  float* part_ml;     // [B, nh, ntiles, 64, 2] per-tile (max, sum) of each row
+  float* row_ml;      // [B, nh, 64, 2] combined (max, 1/sum)
+  float* v_score;     // [B, nh, N]
+  float* dpart;       // [B, nh, ntiles, 192] per-tile diagonal partial sums
+  float* s_score;     // [B, nh, N]
+  DevStatus* status;
+};
+cudaError_t vs_estimate_launch(const VsEstParams& p, cudaStream_t stream);
+
+struct TopkRows {
+  const float* scores;   // row r's scores start at scores + r * row_stride (+ offset)
+  long long row_stride;
+  int rows;              // total rows
+  int len_mode;          // 0: every row has length `len`; 1: row r has length (r % rows_per_group) + 1
+  int len;
+  int rows_per_group;
+  int forced_mode;       // 0: none; 1: index 0; 2: index (r % rows_per_group)
+  int k;
+  int32_t* out_idx;      // [rows, k] ascending, -1 padded
+  int32_t* out_cnt;      // [rows] or NULL
+  DevStatus* status;
+};
+cudaError_t topk_rows_launch(const TopkRows& t, cudaStream_t stream);
+
+struct BsEstParams {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  const int32_t* heads;
+  int nh, B, Hq, Hkv, N, d, group;
+  float scale;
+  float* qbar;     // [B, nh, nb, d]
+  float* kbar;     // [B, nh, nb, d]
+  float* scores;   // [B, nh, nb, nb]
+  DevStatus* status;
+};
+cudaError_t bs_pool_score_launch(const BsEstParams& p, cudaStream_t stream);
+
+struct VsIndexParams {
+  const int32_t* v_idx;
+  const int32_t* s_idx;
+  int nh, B, N, k_v, k_s, wmap_words;
+  minf_vs_index idx;
+  DevStatus* status;
+};
+cudaError_t vs_index_launch(const VsIndexParams& p, cudaStream_t stream);
+
+}  // namespace minf

@@ -1,0 +1,108 @@
+"""One attention layer's pre-fill through libminf: a head -> pattern table
+routes every query head to Vertical-Slash, Block-Sparse or A-shape ("MInference
+1.0" summary, "Summary": a pattern per head chosen offline, indices built
+online, attention over the indices only).
+
+This module only sequences C-ABI calls and owns their buffers (allocated once,
+up front, so that a timed step launches kernels and nothing else).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+from . import minf
+from .workloads import PAT_A, PAT_BS, PAT_VS, Workload
+
+
+@dataclass
+class LayerPlan:
+    w: Workload
+    device: torch.device
+    vs_heads: torch.Tensor | None = None
+    bs_heads: torch.Tensor | None = None
+    a_heads: torch.Tensor | None = None
+    bufs: dict = field(default_factory=dict)
+
+    @property
+    def shape(self):
+        w = self.w
+        return minf.Shape(w.B, w.Hq, w.Hkv, w.N, w.d, 0.0)
+
+
+def make_plan(w: Workload, device="cuda") -> LayerPlan:
+    dev = torch.device(device)
+    plan = LayerPlan(w, dev)
+    shp = plan.shape
+    i32 = dict(dtype=torch.int32, device=dev)
+    vs = w.heads_of(PAT_VS)
+    bs = w.heads_of(PAT_BS)
+    ah = w.heads_of(PAT_A)
+    B, N = w.B, w.N
+    if vs:
+        plan.vs_heads = torch.tensor(vs, **i32)
+        nv = len(vs)
+        plan.bufs["v_idx"] = torch.empty(B, nv, w.k_v, **i32)
+        plan.bufs["s_idx"] = torch.empty(B, nv, w.k_s, **i32)
+        plan.bufs["ws_vs_est"] = minf.workspace(minf.OP_ESTIMATE_VS, shp, nv, device=dev)
+        plan.bufs["ws_vs_idx"] = minf.workspace(minf.OP_BUILD_INDEX, shp, nv, device=dev)
+        plan.bufs["ws_vs_attn"] = minf.workspace(minf.OP_SPARSE_ATTN_VS, shp, nv, device=dev)
+        plan.bufs["vs_index"] = minf.VSIndex.empty(B, nv, N, w.k_v, w.k_s, device=dev)
+    if bs:
+        plan.bs_heads = torch.tensor(bs, **i32)
+        nbh = len(bs)
+        plan.bufs["blk_idx"] = torch.empty(B, nbh, N // 64, w.k_b, **i32)
+        plan.bufs["blk_cnt"] = torch.empty(B, nbh, N // 64, **i32)
+        plan.bufs["ws_bs_est"] = minf.workspace(minf.OP_ESTIMATE_BS, shp, nbh, device=dev)
+        plan.bufs["ws_bs_attn"] = minf.workspace(minf.OP_SPARSE_ATTN_BS, shp, nbh, device=dev)
+    if ah:
+        plan.a_heads = torch.tensor(ah, **i32)
+        plan.bufs["ws_a"] = minf.workspace(minf.OP_ATTN_ASHAPE, shp, len(ah), device=dev)
+    return plan
+
+
+def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None):
+    """Estimation, index build and sparse attention for every head of the
+    layer, in stream order; O (and LSE) are filled head by head."""
+    w, b = plan.w, plan.bufs
+    shp = plan.shape
+    L = minf.lib()
+    st = minf._stream(stream)
+    P = minf._p
+    if plan.vs_heads is not None:
+        nv = plan.vs_heads.numel()
+        minf._check("minf_estimate_vs", L.minf_estimate_vs(
+            minf.ctypes.byref(shp), P(q), P(k), P(plan.vs_heads), nv, w.last_q, w.k_v, w.k_s,
+            P(b["v_idx"]), P(b["s_idx"]), None, None, P(b["ws_vs_est"]), b["ws_vs_est"].numel(), st))
+        ic = b["vs_index"].c()
+        minf._check("minf_build_index", L.minf_build_index(
+            minf.ctypes.byref(shp), nv, P(b["v_idx"]), w.k_v, P(b["s_idx"]), w.k_s, minf.ctypes.byref(ic),
+            P(b["ws_vs_idx"]), b["ws_vs_idx"].numel(), st))
+        minf._check("minf_sparse_attn_vs", L.minf_sparse_attn_vs(
+            minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.vs_heads), nv, minf.ctypes.byref(ic),
+            w.k_v, w.k_s, P(o), P(lse), P(b["ws_vs_attn"]), b["ws_vs_attn"].numel(), st))
+    if plan.bs_heads is not None:
+        nbh = plan.bs_heads.numel()
+        minf._check("minf_estimate_bs", L.minf_estimate_bs(
+            minf.ctypes.byref(shp), P(q), P(k), P(plan.bs_heads), nbh, w.block, w.k_b,
+            P(b["blk_idx"]), P(b["blk_cnt"]), None, P(b["ws_bs_est"]), b["ws_bs_est"].numel(), st))
+        minf._check("minf_sparse_attn_bs", L.minf_sparse_attn_bs(
+            minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.bs_heads), nbh, P(b["blk_idx"]),
+            P(b["blk_cnt"]), w.k_b, P(o), P(lse), P(b["ws_bs_attn"]), b["ws_bs_attn"].numel(), st))
+    if plan.a_heads is not None:
+        na = plan.a_heads.numel()
+        minf._check("minf_attn_ashape", L.minf_attn_ashape(
+            minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.a_heads), na, w.n_sink, w.n_local,
+            P(o), P(lse), P(b["ws_a"]), b["ws_a"].numel(), st))
+    return o, lse
+
+
+def device_status(plan: LayerPlan):
+    """First device-side error code across the plan's workspaces (0 = none)."""
+    for name, t in plan.bufs.items():
+        if name.startswith("ws_"):
+            code = minf.minf_get_device_status(t)
+            if code:
+                return code
+    return 0

@@ -1,0 +1,258 @@
+"""Thin ctypes binding of libminf.so (the C ABI declared in include/minf.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  torch provides device memory and the current stream.  There is no
+CPU fallback: if the library is missing, loading fails with an error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libminf.so")
+
+OK = 0
+STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error",
+                4: "workspace too small", 5: "device timeout", 6: "device bounds"}
+OP_ESTIMATE_VS, OP_ESTIMATE_BS, OP_BUILD_INDEX, OP_SPARSE_ATTN_VS, OP_SPARSE_ATTN_BS, \
+    OP_ATTN_ASHAPE, OP_DENSE_ATTN = range(7)
+
+EXPORTS = ["minf_vs_wmap_words", "minf_workspace_size", "minf_estimate_vs", "minf_estimate_bs",
+           "minf_build_index", "minf_sparse_attn_vs", "minf_sparse_attn_bs", "minf_attn_ashape",
+           "minf_dense_attn", "minf_get_device_status", "minf_status_string"]
+
+
+class MinfError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(code, code)} ({code})")
+        self.code = code
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("N", ctypes.c_int), ("d", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+class _VsIndexC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("grp", "grp_cnt", "tgrp", "tgrp_cnt", "wmap", "vcnt", "vidx")]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libminf.so not found at {LIB_PATH}: run "
+                               "`python -m dynamic_sparse_attention_minf_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, sz, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_int
+        sp = ctypes.POINTER(Shape)
+        L.minf_vs_wmap_words.argtypes = [i]
+        L.minf_vs_wmap_words.restype = sz
+        L.minf_workspace_size.argtypes = [i, sp, i, i, i, i]
+        L.minf_workspace_size.restype = sz
+        L.minf_estimate_vs.argtypes = [sp, vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp]
+        L.minf_estimate_bs.argtypes = [sp, vp, vp, vp, i, i, i, vp, vp, vp, vp, sz, vp]
+        L.minf_build_index.argtypes = [sp, i, vp, i, vp, i, ctypes.POINTER(_VsIndexC), vp, sz, vp]
+        L.minf_sparse_attn_vs.argtypes = [sp, vp, vp, vp, vp, i, ctypes.POINTER(_VsIndexC), i, i,
+                                          vp, vp, vp, sz, vp]
+        L.minf_sparse_attn_bs.argtypes = [sp, vp, vp, vp, vp, i, vp, vp, i, vp, vp, vp, sz, vp]
+        L.minf_attn_ashape.argtypes = [sp, vp, vp, vp, vp, i, i, i, vp, vp, vp, sz, vp]
+        L.minf_dense_attn.argtypes = [sp, vp, vp, vp, vp, i, vp, vp, vp, sz, vp]
+        L.minf_get_device_status.argtypes = [vp, vp]
+        L.minf_status_string.argtypes = [st]
+        L.minf_status_string.restype = ctypes.c_char_p
+        for fn in ("minf_estimate_vs", "minf_estimate_bs", "minf_build_index", "minf_sparse_attn_vs",
+                   "minf_sparse_attn_bs", "minf_attn_ashape", "minf_dense_attn", "minf_get_device_status"):
+            getattr(L, fn).restype = st
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, code):
+    if code != OK:
+        raise MinfError(fn, code)
+
+
+def shape_of(q, k, scale=0.0):
+    B, Hq, N, d = q.shape
+    return Shape(B, Hq, k.shape[1], N, d, float(scale))
+
+
+def workspace(op, shape, nh, k_v=0, k_s=0, k_b=0, device="cuda"):
+    """A zeroed workspace of the size the library asks for."""
+    n = lib().minf_workspace_size(op, ctypes.byref(shape), nh, k_v, k_s, k_b)
+    if n == 0:
+        raise MinfError("minf_workspace_size", 1)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def _heads(heads, device):
+    if heads is None:
+        return None
+    if isinstance(heads, torch.Tensor):
+        return heads.to(device=device, dtype=torch.int32).contiguous()
+    return torch.tensor(list(heads), dtype=torch.int32, device=device)
+
+
+@dataclass
+class VSIndex:
+    """Device buffers of the compact Vertical-Slash index (see minf_vs_index)."""
+    grp: torch.Tensor
+    grp_cnt: torch.Tensor
+    tgrp: torch.Tensor
+    tgrp_cnt: torch.Tensor
+    wmap: torch.Tensor
+    vcnt: torch.Tensor
+    vidx: torch.Tensor
+    k_v: int
+    k_s: int
+
+    @staticmethod
+    def empty(B, nh, N, k_v, k_s, device="cuda"):
+        i32 = dict(dtype=torch.int32, device=device)
+        W = lib().minf_vs_wmap_words(N)
+        return VSIndex(torch.empty(B, nh, k_s, 2, **i32), torch.empty(B, nh, **i32),
+                       torch.empty(B, nh, k_s, 2, **i32), torch.empty(B, nh, **i32),
+                       torch.empty(B, nh, W, **i32), torch.empty(B, nh, N // 64, **i32),
+                       torch.empty(B, nh, N // 64, k_v, **i32), k_v, k_s)
+
+    def c(self):
+        return _VsIndexC(*(t.data_ptr() for t in (self.grp, self.grp_cnt, self.tgrp, self.tgrp_cnt,
+                                                  self.wmap, self.vcnt, self.vidx)))
+
+
+# ----------------------------------------------------------------- entry points
+def minf_estimate_vs(q, k, heads, k_v, k_s, last_q=64, scale=0.0, return_scores=False,
+                     ws=None, stream=None):
+    shp = shape_of(q, k, scale)
+    hd = _heads(heads, q.device)
+    nh = hd.numel()
+    B, N = shp.B, shp.N
+    v_idx = torch.empty(B, nh, k_v, dtype=torch.int32, device=q.device)
+    s_idx = torch.empty(B, nh, k_s, dtype=torch.int32, device=q.device)
+    vs = ss = None
+    if return_scores:
+        vs = torch.empty(B, nh, N, dtype=torch.float32, device=q.device)
+        ss = torch.empty(B, nh, N, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(OP_ESTIMATE_VS, shp, nh, device=q.device)
+    _check("minf_estimate_vs", lib().minf_estimate_vs(
+        ctypes.byref(shp), _p(q), _p(k), _p(hd), nh, last_q, k_v, k_s, _p(v_idx), _p(s_idx),
+        _p(vs), _p(ss), _p(ws), ws.numel(), _stream(stream)))
+    return (v_idx, s_idx, vs, ss) if return_scores else (v_idx, s_idx)
+
+
+def minf_estimate_bs(q, k, heads, k_b, block=64, scale=0.0, return_scores=False, ws=None, stream=None):
+    shp = shape_of(q, k, scale)
+    hd = _heads(heads, q.device)
+    nh = hd.numel()
+    nb = shp.N // 64
+    blk_idx = torch.empty(shp.B, nh, nb, k_b, dtype=torch.int32, device=q.device)
+    blk_cnt = torch.empty(shp.B, nh, nb, dtype=torch.int32, device=q.device)
+    sc = torch.empty(shp.B, nh, nb, nb, dtype=torch.float32, device=q.device) if return_scores else None
+    if ws is None:
+        ws = workspace(OP_ESTIMATE_BS, shp, nh, device=q.device)
+    _check("minf_estimate_bs", lib().minf_estimate_bs(
+        ctypes.byref(shp), _p(q), _p(k), _p(hd), nh, block, k_b, _p(blk_idx), _p(blk_cnt), _p(sc),
+        _p(ws), ws.numel(), _stream(stream)))
+    return (blk_idx, blk_cnt, sc) if return_scores else (blk_idx, blk_cnt)
+
+
+def minf_build_index(shape: Shape, v_idx, s_idx, index: VSIndex | None = None, ws=None, stream=None):
+    B, nh, k_v = v_idx.shape
+    k_s = s_idx.shape[2]
+    if index is None:
+        index = VSIndex.empty(B, nh, shape.N, k_v, k_s, device=v_idx.device)
+    if ws is None:
+        ws = workspace(OP_BUILD_INDEX, shape, nh, device=v_idx.device)
+    ic = index.c()
+    _check("minf_build_index", lib().minf_build_index(
+        ctypes.byref(shape), nh, _p(v_idx), k_v, _p(s_idx), k_s, ctypes.byref(ic), _p(ws), ws.numel(),
+        _stream(stream)))
+    return index
+
+
+def _out(q, o, lse, want_lse):
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    return o, lse
+
+
+def minf_sparse_attn_vs(q, k, v, heads, index: VSIndex, o=None, lse=None, want_lse=True, scale=0.0,
+                        ws=None, stream=None):
+    shp = shape_of(q, k, scale)
+    hd = _heads(heads, q.device)
+    nh = hd.numel()
+    o, lse = _out(q, o, lse, want_lse)
+    if ws is None:
+        ws = workspace(OP_SPARSE_ATTN_VS, shp, nh, device=q.device)
+    ic = index.c()
+    _check("minf_sparse_attn_vs", lib().minf_sparse_attn_vs(
+        ctypes.byref(shp), _p(q), _p(k), _p(v), _p(hd), nh, ctypes.byref(ic), index.k_v, index.k_s,
+        _p(o), _p(lse), _p(ws), ws.numel(), _stream(stream)))
+    return o, lse
+
+
+def minf_sparse_attn_bs(q, k, v, heads, blk_idx, blk_cnt, o=None, lse=None, want_lse=True, scale=0.0,
+                        ws=None, stream=None):
+    shp = shape_of(q, k, scale)
+    hd = _heads(heads, q.device)
+    nh = hd.numel()
+    o, lse = _out(q, o, lse, want_lse)
+    if ws is None:
+        ws = workspace(OP_SPARSE_ATTN_BS, shp, nh, device=q.device)
+    _check("minf_sparse_attn_bs", lib().minf_sparse_attn_bs(
+        ctypes.byref(shp), _p(q), _p(k), _p(v), _p(hd), nh, _p(blk_idx), _p(blk_cnt), blk_idx.shape[-1],
+        _p(o), _p(lse), _p(ws), ws.numel(), _stream(stream)))
+    return o, lse
+
+
+def minf_attn_ashape(q, k, v, heads, n_sink, n_local, o=None, lse=None, want_lse=True, scale=0.0,
+                     ws=None, stream=None):
+    shp = shape_of(q, k, scale)
+    hd = _heads(heads, q.device)
+    nh = hd.numel()
+    o, lse = _out(q, o, lse, want_lse)
+    if ws is None:
+        ws = workspace(OP_ATTN_ASHAPE, shp, nh, device=q.device)
+    _check("minf_attn_ashape", lib().minf_attn_ashape(
+        ctypes.byref(shp), _p(q), _p(k), _p(v), _p(hd), nh, n_sink, n_local, _p(o), _p(lse),
+        _p(ws), ws.numel(), _stream(stream)))
+    return o, lse
+
+
+def minf_dense_attn(q, k, v, heads=None, o=None, lse=None, want_lse=True, scale=0.0, ws=None, stream=None):
+    shp = shape_of(q, k, scale)
+    hd = _heads(heads, q.device)
+    nh = hd.numel() if hd is not None else shp.Hq
+    o, lse = _out(q, o, lse, want_lse)
+    if ws is None:
+        ws = workspace(OP_DENSE_ATTN, shp, nh, device=q.device)
+    _check("minf_dense_attn", lib().minf_dense_attn(
+        ctypes.byref(shp), _p(q), _p(k), _p(v), _p(hd), nh, _p(o), _p(lse), _p(ws), ws.numel(),
+        _stream(stream)))
+    return o, lse
+
+
+def minf_get_device_status(ws, stream=None):
+    return lib().minf_get_device_status(_p(ws), _stream(stream))

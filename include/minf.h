@@ -1,0 +1,214 @@
+/*
+ * minf.h -- C ABI of libminf.so: the pre-fill hot path of dynamic sparse
+ * attention ("MInference 1.0: Accelerating Pre-filling for Long-Context LLMs
+ * via Dynamic Sparse Attention"), built for NVIDIA B200 (sm_100a).
+ *
+ * The method (abstract; summary page, "Summary" and "Key points"): every
+ * attention head follows one of three patterns -- A-shape, Vertical-Slash or
+ * Block-Sparse.  At inference time the sparse indices of a Vertical-Slash
+ * head are estimated by scoring the last query vectors against all keys, and
+ * those of a Block-Sparse head from queries and keys mean-pooled in 64-token
+ * blocks; attention is then computed over those indices only.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are dense, row-major, on the device, owned by the caller:
+ *      Q, O : [B, Hq,  N, d]  bf16 (raw bits, minf_bf16)
+ *      K, V : [B, Hkv, N, d]  bf16
+ *      LSE  : [B, Hq,  N]     fp32, natural-log log-sum-exp of each row
+ *    Query head h reads KV head h / (Hq / Hkv) (grouped-query attention).
+ *  - `heads` is a device array of `nh` query-head ids (int32, each in
+ *    [0, Hq), no duplicates).  Per-head index arrays are laid out [B, nh, ...]
+ *    in the order of that list.  Attention calls write O (and LSE) only for
+ *    the listed heads, so calls for different patterns fill disjoint heads of
+ *    one O.  Where documented, heads == NULL means all Hq heads (nh = Hq).
+ *  - Requirements: N % 128 == 0, d in {64, 128}, Hq % Hkv == 0, B >= 1.  Violations return MINF_ERR_INVALID_ARG or MINF_ERR_UNSUPPORTED
+ *    before anything is launched.
+ *  - The library allocates no device memory.  Scratch space comes from the
+ *    caller's workspace `ws` of `ws_bytes` bytes, sized by
+ *    minf_workspace_size(); its first 256 bytes hold a device status word
+ *    that kernels set on a device-side error (a bounded wait that ran out,
+ *    an index out of range).  Zero the workspace once before first use;
+ *    read and clear the status with minf_get_device_status().
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and returns a host-side status: launch errors
+ *    come back as MINF_ERR_CUDA.
+ *  - Selection ties go to the lower index; selected index lists are sorted
+ *    ascending.  A requested k larger than the number of candidates is
+ *    clamped to it.
+ */
+#ifndef MINF_H
+#define MINF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t minf_bf16; /* raw bfloat16 bits */
+
+typedef enum {
+  MINF_OK = 0,
+  MINF_ERR_INVALID_ARG = 1,
+  MINF_ERR_UNSUPPORTED = 2,
+  MINF_ERR_CUDA = 3,
+  MINF_ERR_WORKSPACE_TOO_SMALL = 4,
+  MINF_ERR_DEVICE_TIMEOUT = 5,   /* a kernel's bounded wait expired; outputs are invalid */
+  MINF_ERR_DEVICE_BOUNDS = 6     /* a kernel found an index outside its range; outputs are invalid */
+} minf_status;
+
+/* Problem geometry.  scale <= 0 selects the softmax temperature 1/sqrt(d). */
+typedef struct {
+  int B, Hq, Hkv, N, d;
+  float scale;
+} minf_shape;
+
+/* Operation ids for minf_workspace_size(). */
+enum {
+  MINF_OP_ESTIMATE_VS = 0,
+  MINF_OP_ESTIMATE_BS = 1,
+  MINF_OP_BUILD_INDEX = 2,
+  MINF_OP_SPARSE_ATTN_VS = 3,
+  MINF_OP_SPARSE_ATTN_BS = 4,
+  MINF_OP_ATTN_ASHAPE = 5,
+  MINF_OP_DENSE_ATTN = 6
+};
+
+/*
+ * Compact Vertical-Slash index of nh heads, written by minf_build_index and
+ * read by minf_sparse_attn_vs.  All buffers are caller-owned device memory;
+ * nb = N / 64, W = minf_vs_wmap_words(N).
+ *   grp      [B, nh, k_s, 2] slash groups (a_g, b_g): ascending offsets merged
+ *                            while consecutive offsets differ by <= 64
+ *   grp_cnt  [B, nh]         number of groups
+ *   tgrp     [B, nh, k_s, 2] the same offsets merged while they differ by
+ *                            <= 128 (the bands of a 128-row query tile)
+ *   tgrp_cnt [B, nh]
+ *   wmap     [B, nh, W]      bit x set iff block offset u = x - 63 lies in
+ *                            some [a_g - 63, b_g]: key j is on a slash band of
+ *                            the query block whose first row is r0 exactly
+ *                            when bit (r0 - j + 63) is set
+ *   vcnt     [B, nh, nb]     per 64-row query block, the number of vertical
+ *                            columns not already covered by a slash band
+ *   vidx     [B, nh, nb, k_v] those columns, ascending (j <= last row of the block)
+ */
+typedef struct {
+  int32_t* grp;
+  int32_t* grp_cnt;
+  int32_t* tgrp;
+  int32_t* tgrp_cnt;
+  uint32_t* wmap;
+  int32_t* vcnt;
+  int32_t* vidx;
+} minf_vs_index;
+
+/* Number of 32-bit words of one head's slash-band bitmap (wmap). */
+size_t minf_vs_wmap_words(int N);
+
+/*
+ * Bytes of workspace that operation `op` needs for this shape, head count and
+ * budgets (k_v, k_s, k_b are ignored where the operation has none).  Always at
+ * least 256 (the status word).  Returns 0 for an unknown op or a bad shape.
+ */
+size_t minf_workspace_size(int op, const minf_shape* shape, int nh, int k_v, int k_s, int k_b);
+
+/*
+ * Vertical-Slash index estimation (summary, "Key points": the last query
+ * vectors are scored against all keys).  For each listed head and each of
+ * the last `last_q` query rows i (1 <= last_q <= 64; the pages' reading is
+ * 64), the causal scores s_ij = scale * q_i . k_j (j <= i) are softmax-ed
+ * over j in fp32; then
+ *     v_j     = sum_i p_ij           (vertical score of key column j)
+ *     sigma_o = sum_i p_{i, i-o}     (slash score of diagonal offset o >= 0)
+ * v_idx gets the k_v best columns, s_idx the k_s best offsets with offset 0
+ * always kept; both ascending.  v_score / s_score ([B, nh, N] fp32) receive
+ * the scores when non-NULL.  Outputs: v_idx [B, nh, k_v], s_idx [B, nh, k_s].
+ */
+minf_status minf_estimate_vs(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K,
+                             const int32_t* heads, int nh, int last_q, int k_v, int k_s,
+                             int32_t* v_idx, int32_t* s_idx, float* v_score, float* s_score,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Block-Sparse index estimation (summary, "Key points": queries and keys are
+ * mean-pooled in 64-token blocks).  Pooled means are taken in fp32 and the
+ * pooled scores t[b, c] = scale * Qbar_b . Kbar_c (c <= b) are formed with fp32
+ * FMAs; per query block b the k_b best key blocks are kept, block b itself
+ * always.  block must be 64.  Outputs: blk_idx [B, nh, N/64, k_b] ascending,
+ * padded with -1; blk_cnt [B, nh, N/64] = min(b + 1, k_b).  blk_score, when
+ * non-NULL, receives t as [B, nh, N/64, N/64] (entries with c > b undefined).
+ */
+minf_status minf_estimate_bs(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K,
+                             const int32_t* heads, int nh, int block, int k_b,
+                             int32_t* blk_idx, int32_t* blk_cnt, float* blk_score,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Vertical-Slash index build: compacts v_idx [B, nh, k_v] and s_idx
+ * [B, nh, k_s] (both ascending, as minf_estimate_vs writes them) into the
+ * minf_vs_index above.  A slash offset o covers, in a 64-row query block with
+ * first row r0, the keys r0 - o .. r0 + 63 - o; verticals already on such a
+ * band are dropped from that block's list so that every key is counted once.
+ * Unsorted or out-of-range input indices set MINF_ERR_DEVICE_BOUNDS.
+ */
+minf_status minf_build_index(const minf_shape* shape, int nh, const int32_t* v_idx, int k_v,
+                             const int32_t* s_idx, int k_s, const minf_vs_index* idx,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Vertical-Slash sparse attention (summary, "Summary", stage 3: attention
+ * over the estimated indices only).  Row i of query block b attends to the
+ * keys j <= i that lie on a slash band of block b or in block b's vertical
+ * list; softmax in fp32, P.V in bf16 with fp32 accumulation, on tcgen05
+ * tensor cores.  lse may be NULL.
+ */
+minf_status minf_sparse_attn_vs(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K,
+                                const minf_bf16* V, const int32_t* heads, int nh,
+                                const minf_vs_index* idx, int k_v, int k_s,
+                                minf_bf16* O, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Block-Sparse sparse attention: row i attends to keys j <= i whose 64-key
+ * block is listed for i's query block in blk_idx / blk_cnt (as written by
+ * minf_estimate_bs).  lse may be NULL.
+ */
+minf_status minf_sparse_attn_bs(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K,
+                                const minf_bf16* V, const int32_t* heads, int nh,
+                                const int32_t* blk_idx, const int32_t* blk_cnt, int k_b,
+                                minf_bf16* O, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * A-shape attention (abstract; summary, "Summary": the A-shape pattern):
+ * row i attends to keys j <= i with j < n_sink or i - j < n_local.  lse may be
+ * NULL.  n_sink >= 0, n_local >= 1.
+ */
+minf_status minf_attn_ashape(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K,
+                             const minf_bf16* V, const int32_t* heads, int nh, int n_sink,
+                             int n_local, minf_bf16* O, float* lse, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/*
+ * Dense causal attention (the baseline the pages' speed-ups are measured
+ * against; summary, "Key points": the kernels build on FlashAttention), on
+ * the same tcgen05 mainloop.  heads may be NULL (all heads).  lse may be NULL.
+ */
+minf_status minf_dense_attn(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K,
+                            const minf_bf16* V, const int32_t* heads, int nh, minf_bf16* O,
+                            float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronizes `stream`, returns the device status word of `ws` (MINF_OK when
+ * no kernel reported an error since the last call) and clears it.
+ */
+minf_status minf_get_device_status(void* ws, void* stream);
+
+/* Static description of a status code. */
+const char* minf_status_string(minf_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MINF_H */

@@ -1,0 +1,192 @@
+"""GPU parity: every C-ABI entry point against the CPU oracle on the same
+seeded bf16 inputs (indices bit-exact up to the score-gap rule, attention
+within max-abs 2e-2 / mean-abs 2e-3)."""
+import numpy as np
+import pytest
+import torch
+
+from dynamic_sparse_attention_minf_b200 import minf
+from dynamic_sparse_attention_minf_b200 import workloads as wl
+from oracle import minf_oracle as orc
+from tests.parity import check_close, check_index_set, check_lse
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    minf.lib()
+
+
+def _inputs(w):
+    q, k, v = wl.make_qkv(w, DEV)
+    return q, k, v, orc.to_f64(q[0]), orc.to_f64(k[0]), orc.to_f64(v[0])
+
+
+def _check_attn(o, lse, qn, kn, vn, heads, w, mask_for_head, rows=None):
+    N = w.N
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    sc = orc.default_scale(w.d)
+    on = o[0].float().cpu().numpy()
+    ln = lse[0].cpu().numpy()
+    for hi, h in enumerate(heads):
+        kv = orc.kv_head(h, w.Hq, w.Hkv)
+        O, L = orc.attention_head(qn[h], kn[kv], vn[kv], rows, mask_for_head(hi, h), sc)
+        check_close(on[h][rows], O, f"head {h}")
+        check_lse(ln[h][rows], L, f"head {h}")
+
+
+# ------------------------------------------------------------------ dense
+@pytest.mark.parametrize("Hq,Hkv,N,d", [(2, 1, 512, 64), (2, 2, 1024, 128), (4, 2, 640, 128)])
+def test_dense_attention(Hq, Hkv, N, d):
+    w = wl.small(Hq=Hq, Hkv=Hkv, N=N, d=d, seed=N + d)
+    q, k, v, qn, kn, vn = _inputs(w)
+    ws = minf.workspace(minf.OP_DENSE_ATTN, minf.shape_of(q, k), Hq)
+    o, lse = minf.minf_dense_attn(q, k, v, ws=ws)
+    assert minf.minf_get_device_status(ws) == 0
+    _check_attn(o, lse, qn, kn, vn, range(Hq), w, lambda hi, h: (lambda r: orc.mask_dense(r, N)))
+
+
+# ---------------------------------------------------------------- A-shape
+@pytest.mark.parametrize("n_sink,n_local,N,d", [(64, 300, 1024, 128), (100, 129, 768, 64), (0, 64, 512, 128),
+                                                (128, 4096, 1024, 128)])
+def test_ashape_attention(n_sink, n_local, N, d):
+    w = wl.small(Hq=4, Hkv=2, N=N, d=d, seed=3 + n_local)
+    q, k, v, qn, kn, vn = _inputs(w)
+    heads = [1, 2]
+    ws = minf.workspace(minf.OP_ATTN_ASHAPE, minf.shape_of(q, k), 2)
+    o, lse = minf.minf_attn_ashape(q, k, v, heads, n_sink, n_local, ws=ws)
+    assert minf.minf_get_device_status(ws) == 0
+    _check_attn(o, lse, qn, kn, vn, heads, w,
+                lambda hi, h: (lambda r: orc.mask_ashape(r, N, n_sink, n_local)))
+
+
+# --------------------------------------------------------- Vertical-Slash
+def _vs_pipeline(w, heads, rows=None):
+    q, k, v, qn, kn, vn = _inputs(w)
+    sc = orc.default_scale(w.d)
+    ws = minf.workspace(minf.OP_ESTIMATE_VS, minf.shape_of(q, k), len(heads))
+    v_idx, s_idx, vs, ss = minf.minf_estimate_vs(q, k, heads, w.k_v, w.k_s, return_scores=True, ws=ws)
+    assert minf.minf_get_device_status(ws) == 0
+    gv, gs = v_idx[0].cpu().numpy(), s_idx[0].cpu().numpy()
+    for hi, h in enumerate(heads):
+        kv = orc.kv_head(h, w.Hq, w.Hkv)
+        rv, rs = orc.vs_estimate(qn[h][w.N - 64:], kn[kv], sc)
+        np.testing.assert_allclose(vs[0, hi].cpu().numpy(), rv, rtol=1e-4, atol=1e-7)
+        np.testing.assert_allclose(ss[0, hi].cpu().numpy(), rs, rtol=1e-4, atol=1e-7)
+        ov, os_ = orc.vs_select(rv, rs, w.k_v, w.k_s)
+        check_index_set(gv[hi], ov, rv, what=f"vertical h{h}")
+        check_index_set(gs[hi], os_, rs, forced=0, what=f"slash h{h}")
+    index = minf.minf_build_index(minf.shape_of(q, k), v_idx, s_idx)
+    o, lse = minf.minf_sparse_attn_vs(q, k, v, heads, index)
+    torch.cuda.synchronize()
+    # index build is integer work: bit-exact against the oracle on the GPU's own V and S
+    for hi in range(len(heads)):
+        groups, vcnt, vidx = orc.vs_build_index(gv[hi], gs[hi], w.N)
+        G = int(index.grp_cnt[0, hi])
+        assert G == groups.shape[0]
+        assert np.array_equal(index.grp[0, hi, :G].cpu().numpy(), groups)
+        tg = orc.vs_groups(gs[hi], block=128)
+        T = int(index.tgrp_cnt[0, hi])
+        assert T == tg.shape[0] and np.array_equal(index.tgrp[0, hi, :T].cpu().numpy(), tg)
+        assert np.array_equal(index.vcnt[0, hi].cpu().numpy(), vcnt)
+        gvi = index.vidx[0, hi].cpu().numpy()
+        for b in range(w.N // 64):
+            assert np.array_equal(gvi[b, :vcnt[b]], vidx[b, :vcnt[b]]), f"block {b}"
+    _check_attn(o, lse, qn, kn, vn, heads, w,
+                lambda hi, h: (lambda r: orc.mask_vs(r, w.N, gv[hi], gs[hi])), rows)
+    return gv, gs
+
+
+def test_vs_pipeline_small():
+    w = wl.small(Hq=4, Hkv=2, N=2048, d=128, seed=21, k_v=64, k_s=128)
+    _vs_pipeline(w, [0, 3])
+
+
+def test_vs_config0():
+    """Vertical-Slash, H=1, N=4096, d=64, vertical 128 / slash 256, sink bias."""
+    w = wl.config(0)
+    _vs_pipeline(w, [0])
+
+
+def test_vs_all_selected_equals_dense():
+    """Closed form: with every column and every offset kept, VS is dense causal."""
+    w = wl.small(Hq=2, Hkv=1, N=512, d=64, seed=5, k_v=512, k_s=512)
+    q, k, v, *_ = _inputs(w)
+    v_idx, s_idx = minf.minf_estimate_vs(q, k, [0, 1], 512, 512)
+    assert torch.equal(v_idx[0, 0].cpu(), torch.arange(512, dtype=torch.int32))
+    index = minf.minf_build_index(minf.shape_of(q, k), v_idx, s_idx)
+    o, lse = minf.minf_sparse_attn_vs(q, k, v, [0, 1], index)
+    od, ld = minf.minf_dense_attn(q, k, v)
+    assert (o.float() - od.float()).abs().max().item() <= 1e-2
+    assert (lse - ld).abs().max().item() <= 1e-3
+
+
+def test_vs_index_from_oracle_sets():
+    """build_index + attention on oracle-chosen sets with wide gaps and long groups."""
+    w = wl.small(Hq=2, Hkv=1, N=4096, d=128, seed=8, k_v=300, k_s=700)
+    q, k, v, qn, kn, vn = _inputs(w)
+    rng = np.random.default_rng(0)
+    S = np.unique(np.concatenate([[0], np.arange(1, 400), rng.choice(4096, 400, replace=False)]))[:700]
+    V = np.unique(rng.choice(4096, 300, replace=False))
+    assert S.size == 700 and V.size == 300
+    v_idx = torch.tensor(np.stack([V, V])[None], dtype=torch.int32, device=DEV)
+    s_idx = torch.tensor(np.stack([S, S])[None], dtype=torch.int32, device=DEV)
+    index = minf.minf_build_index(minf.shape_of(q, k), v_idx, s_idx)
+    o, lse = minf.minf_sparse_attn_vs(q, k, v, [0, 1], index)
+    _check_attn(o, lse, qn, kn, vn, [0, 1], w, lambda hi, h: (lambda r: orc.mask_vs(r, w.N, V, S)))
+
+
+# ----------------------------------------------------------- Block-Sparse
+def _bs_pipeline(w, heads, rows=None):
+    q, k, v, qn, kn, vn = _inputs(w)
+    sc = orc.default_scale(w.d)
+    ws = minf.workspace(minf.OP_ESTIMATE_BS, minf.shape_of(q, k), len(heads))
+    blk_idx, blk_cnt, t = minf.minf_estimate_bs(q, k, heads, w.k_b, return_scores=True, ws=ws)
+    assert minf.minf_get_device_status(ws) == 0
+    gi, gc = blk_idx[0].cpu().numpy(), blk_cnt[0].cpu().numpy()
+    nb = w.N // 64
+    flips = 0
+    for hi, h in enumerate(heads):
+        kv = orc.kv_head(h, w.Hq, w.Hkv)
+        ri, rc = orc.bs_select(qn[h], kn[kv], sc, w.k_b)
+        tref = orc.bs_scores(orc.bs_pool(qn[h]), orc.bs_pool(kn[kv]), sc)
+        tg = t[0, hi].cpu().numpy()
+        low = np.tril(np.ones((nb, nb), bool))
+        np.testing.assert_allclose(tg[low], tref[low], rtol=1e-4, atol=1e-5)
+        assert np.array_equal(gc[hi], rc)
+        for b in range(nb):
+            flips += check_index_set(gi[hi, b, :gc[hi, b]], ri[b, :rc[b]], tref[b, :b + 1], forced=b,
+                                     what=f"h{h} block {b}")
+            assert (gi[hi, b, gc[hi, b]:] == -1).all()
+    o, lse = minf.minf_sparse_attn_bs(q, k, v, heads, blk_idx, blk_cnt)
+    torch.cuda.synchronize()
+    _check_attn(o, lse, qn, kn, vn, heads, w,
+                lambda hi, h: (lambda r: orc.mask_bs(r, w.N, gi[hi], gc[hi])), rows)
+    return flips
+
+
+def test_bs_pipeline_small():
+    w = wl.small(Hq=4, Hkv=2, N=2048, d=128, seed=4, bias="block", patterns=[wl.PAT_BS] * 4, k_b=7)
+    _bs_pipeline(w, [1, 2])
+
+
+def test_bs_config1_sampled_rows():
+    """Block-Sparse, 8 heads (MHA), N=32768, d=128, top-64 blocks."""
+    w = wl.config(1)
+    rows = wl.sample_rows(w.N, 512, w.seed).numpy()
+    _bs_pipeline(w, list(range(8)), rows)
+
+
+def test_bs_all_blocks_equals_dense():
+    w = wl.small(Hq=2, Hkv=1, N=1024, d=128, seed=9, bias="block", patterns=[wl.PAT_BS] * 2, k_b=64)
+    q, k, v, *_ = _inputs(w)
+    blk_idx, blk_cnt = minf.minf_estimate_bs(q, k, [0, 1], 64)
+    o, lse = minf.minf_sparse_attn_bs(q, k, v, [0, 1], blk_idx, blk_cnt)
+    od, ld = minf.minf_dense_attn(q, k, v)
+    assert (o.float() - od.float()).abs().max().item() <= 1e-2
+    assert (lse - ld).abs().max().item() <= 1e-3
