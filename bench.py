@@ -1,0 +1,394 @@
+"""Benchmark: one pre-fill attention layer of the 1M-token LLaMA-3-8B-shaped
+workload (32 query / 8 KV heads, d=128, N=1048576; 24 Vertical-Slash heads
+with vertical 2000 / slash 12000, 6 Block-Sparse heads with top-100 blocks,
+2 A-shape heads with 128 sink + 4096 local) through libminf.
+
+A step is the whole hot path for every head: index estimation, index build
+and sparse attention.  ``value`` is the effective throughput: the attention
+work the masks keep (4 d per kept score entry: Q K^T and P V) divided by the
+device time of the step, with inputs already in HBM.  ``e2e`` is the same
+quantity with pinned-host inputs copied in and the output copied out inside
+the timed region.  The roofline object reports the dominant kernel (the
+Vertical-Slash attention launch) against the measured bf16 tensor peak, on
+the tiles it actually executes.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun) every rank runs its own layer (independent prompts, no
+collective on the data path: weak scaling); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+WORKLOAD_ID = 4
+METRIC = "prefill sparse-attention ms and effective TFLOP/s at N=128K–1M, % bf16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}",
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        try:
+            lines = [l.split(",") for l in open(self.path).read().strip().splitlines() if l.strip()]
+        except OSError:
+            return None
+        if not lines:
+            return None
+        mhz = [float(l[1]) for l in lines if l[1].strip().replace(".", "").isdigit()]
+        mx = max(float(l[2]) for l in lines)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for l in lines for i in range(4)
+                          if len(l) > 5 + i and l[5 + i].strip() == "Active"})
+        loaded = [m for m in mhz if m > 0.5 * mx] or mhz
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(lines)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        rank = int(os.environ["RANK"])
+        local = int(os.environ.get("LOCAL_RANK", rank))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, rank, ws, local
+    return None, 0, 1, 0
+
+
+def _max_over_ranks(dist, x: float) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def _counters(ws):
+    c = ws[:24].cpu().view(torch.int64)
+    return int(c[1]), int(c[2])
+
+
+# ----------------------------------------------------------- CPU oracle leg
+def oracle_sample(w, q, k, v, plan, rows_per_pattern=16, seed=0):
+    """The oracle on a bounded sample of the workload: one head of each
+    pattern gets its full index estimation and `rows_per_pattern` sampled
+    query rows of attention.  Returns (useful FLOPs, seconds, seconds per row
+    and per head estimate) so that callers can scale to the whole layer."""
+    import numpy as np
+    from oracle import minf_oracle as orc
+    from dynamic_sparse_attention_minf_b200 import workloads as wl
+
+    sc = orc.default_scale(w.d)
+    rows = wl.sample_rows(w.N, rows_per_pattern, seed).numpy()
+    out = {}
+    for pat in (wl.PAT_VS, wl.PAT_BS, wl.PAT_A):
+        heads = w.heads_of(pat)
+        if not heads:
+            continue
+        h = heads[0]
+        kv = orc.kv_head(h, w.Hq, w.Hkv)
+        kn = orc.to_f64(k[0, kv])
+        vn = orc.to_f64(v[0, kv])
+        qr = orc.to_f64(q[0, h])
+        t0 = time.perf_counter()
+        if pat == wl.PAT_VS:
+            vv, ss = orc.vs_estimate(qr[w.N - w.last_q:], kn, sc)
+            V, S = orc.vs_select(vv, ss, w.k_v, w.k_s)
+            fn = lambda r: orc.mask_vs(r, w.N, V, S)
+        elif pat == wl.PAT_BS:
+            # pooling for the whole head, selection for the sampled rows' query
+            # blocks only (its time is scaled to all blocks below)
+            blks = np.unique(rows // w.block)
+            orc.bs_pool(qr, w.block), orc.bs_pool(kn, w.block)
+            t_pool = time.perf_counter() - t0
+            bi_s, bc_s = orc.bs_select(qr, kn, sc, w.k_b, blocks=blks)
+            nb = w.N // w.block
+            bi = np.full((nb, w.k_b), -1, np.int64)
+            bc = np.zeros(nb, np.int64)
+            bi[blks], bc[blks] = bi_s, bc_s
+            fn = lambda r, bi=bi, bc=bc: orc.mask_bs(r, w.N, bi, bc)
+        else:
+            fn = lambda r: orc.mask_ashape(r, w.N, w.n_sink, w.n_local)
+        t1 = time.perf_counter()
+        if pat == wl.PAT_BS:
+            sel = (t1 - t0) - 2 * t_pool
+            t0 = t1 - (t_pool + max(sel, 0.0) * (w.N // w.block) / len(np.unique(rows // w.block)))
+        nnz = int(fn(rows).sum())
+        orc.attention_head(qr, kn, vn, rows, fn, sc)
+        t2 = time.perf_counter()
+        out[pat] = dict(est_s=t1 - t0, row_s=(t2 - t1) / len(rows), nnz_per_row=nnz / len(rows),
+                        heads=len(heads))
+    # scale to the whole layer: estimation per head + attention per row
+    total_s = sum(o["heads"] * (o["est_s"] + o["row_s"] * w.N) for o in out.values())
+    flops = sum(o["heads"] * 4.0 * w.d * o["nnz_per_row"] * w.N for o in out.values())
+    sample_s = sum(o["est_s"] + o["row_s"] * len(rows) for o in out.values())
+    return flops, total_s, sample_s, out
+
+
+def _cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"), default=1)
+        return int(n)
+    except Exception:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def run_reference(args, dist, rank, world):
+    """The oracle (test infrastructure, as it stands) timed on host cores."""
+    if rank != 0:
+        return
+    from dynamic_sparse_attention_minf_b200 import workloads as wl
+    w = wl.config(WORKLOAD_ID)
+    q, k, v = wl.make_qkv(w, "cuda" if torch.cuda.is_available() else "cpu")
+    times, flops_l, samples = [], [], []
+    for step in range(args.warmup + args.steps):
+        flops, total_s, sample_s, _ = oracle_sample(w, q, k, v, None, rows_per_pattern=8, seed=step)
+        if step >= args.warmup:
+            times.append(total_s)
+            flops_l.append(flops)
+            samples.append(sample_s)
+    val = sum(flops_l) / sum(times) / 1e12
+    ms = 1000.0 * statistics.mean(times)
+    cores = _cores()
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": "per step: one head of each pattern with full index estimation "
+                                       "and 8 sampled query rows, scaled to all heads and rows "
+                                       f"(measured {statistics.mean(samples):.1f} s of CPU per step)"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args, dist, rank, world, local):
+    from dynamic_sparse_attention_minf_b200 import layer, minf
+    from dynamic_sparse_attention_minf_b200 import workloads as wl
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = wl.config(WORKLOAD_ID)
+    w.seed += 100 * rank                      # independent prompts per rank
+    q, k, v = wl.make_qkv(w, dev)
+    plan = layer.make_plan(w, dev)
+    o = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    # one counted run: executed tiles and kept entries per pattern
+    for name in ("ws_vs_attn", "ws_bs_attn", "ws_a"):
+        plan.bufs[name].zero_()
+    layer.run_layer(plan, q, k, v, o)
+    torch.cuda.synchronize()
+    status = layer.device_status(plan)
+    if status:
+        raise RuntimeError(f"device status {status}")
+    cnt = {n: _counters(plan.bufs[n]) for n in ("ws_vs_attn", "ws_bs_attn", "ws_a")}
+    tile_flops = 4.0 * 128 * 128 * w.d
+    useful = sum(4.0 * w.d * c[1] for c in cnt.values())
+    executed = sum(tile_flops * c[0] for c in cnt.values())
+    vs_exec = tile_flops * cnt["ws_vs_attn"][0]
+
+    # warm-up
+    for _ in range(args.warmup):
+        layer.run_layer(plan, q, k, v, o)
+    torch.cuda.synchronize()
+
+    # timed device steps, with events around the VS attention launch
+    marks = []
+
+    class Marks:
+        def mark(self, name):
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            marks.append((name, e))
+
+    mk = Marks()
+    with ClockSampler(local) as clk:
+        time.sleep(1.0)                      # let the sampler start before timing
+        _barrier(dist)
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        ev[0].record(stream)
+        for s_ in range(args.steps):
+            layer.run_layer(plan, q, k, v, o, marks=mk)
+            ev[s_ + 1].record(stream)
+        torch.cuda.synchronize()
+        _barrier(dist)
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    step_ms = ev[0].elapsed_time(ev[-1]) / args.steps
+    step_ms = _max_over_ranks(dist, step_ms)
+    vs_ms = []
+    for a, b in zip(marks[0::2], marks[1::2]):
+        if a[0] == "vs_attn:pre" and b[0] == "vs_attn:post":
+            vs_ms.append(a[1].elapsed_time(b[1]))
+    vs_ms = statistics.mean(vs_ms) if vs_ms else None
+
+    # end to end through the public API: pinned host in, host out
+    hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    hk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+    hv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hq.copy_(q)
+    hk.copy_(k)
+    hv.copy_(v)
+    e2e_steps = max(1, min(args.steps, 3))
+    _barrier(dist)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        layer.run_layer(plan, q, k, v, o)
+        ho.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(dist, e0.elapsed_time(e1) / e2e_steps)
+    h2d = (q.numel() + k.numel() + v.numel()) * 2
+    d2h = o.numel() * 2
+
+    # dense baseline from the same library: one head, scaled to all heads
+    dense_ms = None
+    if rank == 0 and not args.no_dense:
+        od = torch.empty_like(q)
+        wsd = minf.workspace(minf.OP_DENSE_ATTN, plan.shape, 1, device=dev)
+        h0 = torch.tensor([0], dtype=torch.int32, device=dev)
+        minf.minf_dense_attn(q, k, v, h0, o=od, want_lse=False, ws=wsd)
+        torch.cuda.synchronize()
+        d0 = torch.cuda.Event(enable_timing=True)
+        d1 = torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        minf.minf_dense_attn(q, k, v, h0, o=od, want_lse=False, ws=wsd)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = d0.elapsed_time(d1) * w.Hq
+        del od
+
+    if rank != 0:
+        return
+    peaks, src = _peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    achieved = vs_exec / (vs_ms * 1e-3) / 1e12 if vs_ms else None
+    cpu = None
+    if world == 1 and not args.no_cpu:
+        flops_c, total_s, sample_s, _ = oracle_sample(w, q, k, v, plan, rows_per_pattern=96)
+        cpu = {"value": flops_c / total_s / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+               "sample": "one head of each pattern with full index estimation and 96 sampled query rows, "
+                         f"scaled to all heads and rows ({sample_s:.1f} s of CPU)"}
+    clocks = clk.summary()
+    val = world * useful / (step_ms * 1e-3) / 1e12
+    dense_flops = 4.0 * w.d * (w.N * (w.N + 1) / 2) * w.Hq
+    line = {
+        "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+                   "patterns": "24 vertical-slash (2000/12000), 6 block-sparse (top-100), 2 a-shape (128+4096)",
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs 12 GiB per step, larger than the 126 MB L2 (no flush needed)"},
+        "step_ms_each": [round(x, 2) for x in per_step],
+        "useful_tflop_per_step": useful / 1e12, "executed_tflop_per_step": executed / 1e12,
+        "density_vs_dense": useful / dense_flops,
+        "dense_attn_ms_est": dense_ms,
+        "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None,
+        "roofline": {"kernel": "attn_kernel<128, vertical_slash>", "bound": "tensor",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "peak_source": f"{src} bf16_tflops_sustained", "ms_per_launch": vs_ms,
+                     "executed_tflop_per_launch": vs_exec / 1e12},
+        "e2e": {"value": world * useful / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": layer.LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense baseline")
+    args = ap.parse_args()
+    dist, rank, world, local = _dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, dist, rank, world)
+        else:
+            run_ours(args, dist, rank, world, local)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

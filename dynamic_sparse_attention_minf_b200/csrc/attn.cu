@@ -549,6 +549,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     __syncwarp();
     produce_tiles<D, POL>(P, p, b, hi, qt);
+    if (lane == 0 && P.ok) atomicAdd(&p.status->tiles, (unsigned long long)P.t);
     P.emit_end();
     P.flush_pending();
     P.drain();
@@ -615,6 +616,7 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t srow = tmem + ((uint32_t)(q4 * 32) << 16);
     float m_run = -INFINITY, l_run = 0.f;
     int n = 0;
+    unsigned nnz = 0;
     for (int t = wg;; t += 2) {
       const int st = t % C::kStages;
       if (!warp_wait(&k_full[st], (t / C::kStages) & 1, abort, p.status, 10)) break;
@@ -634,6 +636,11 @@ __global__ void __launch_bounds__(320, 1)
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
 
       const int flags = dd.flags;
+      if (!(flags & (F_CAUSAL | F_ASHAPE))) {
+        nnz += (flags & F_MASK) ? __popc(dd.mask[half][0]) + __popc(dd.mask[half][1]) +
+                                      __popc(dd.mask[half][2]) + __popc(dd.mask[half][3])
+                                : 128u;
+      }
       if (flags & F_MASK) {
         const uint32_t mw0 = dd.mask[half][0], mw1 = dd.mask[half][1];
         const uint32_t mw2 = dd.mask[half][2], mw3 = dd.mask[half][3];
@@ -662,6 +669,10 @@ __global__ void __launch_bounds__(320, 1)
             if (causal && j > i) s[c] = -INFINITY;
           }
         }
+      }
+      if (flags & (F_CAUSAL | F_ASHAPE)) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) nnz += (s[c] != -INFINITY);
       }
       float mx = -INFINITY;
 #pragma unroll
@@ -711,6 +722,12 @@ __global__ void __launch_bounds__(320, 1)
       ++n;
     }
     // ----------------------------------------------------------- epilogue
+    {
+      unsigned long long c = nnz;
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+      if (lane == 0) atomicAdd(&p.status->nnz, c);
+    }
     bool ok = !*abort;
     if (ok && n > 0) ok = warp_wait(&o_done[wg], (n - 1) & 1, abort, p.status, 13);
     named_bar_sync(1, 256);

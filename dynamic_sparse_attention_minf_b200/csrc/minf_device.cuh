@@ -15,10 +15,13 @@ namespace minf {
 
 // ---------------------------------------------------------------- status word
 // The first 256 bytes of every workspace: word 0 holds the first device error
-// code (MINF_ERR_DEVICE_*), word 1 a detail code of where it happened.
+// code (MINF_ERR_DEVICE_*), word 1 a detail code of where it happened; the
+// attention kernels also accumulate two work counters there.
 struct DevStatus {
   int code;
   int where;
+  unsigned long long tiles;  // attention: 128 x 128 key tiles executed
+  unsigned long long nnz;    // attention: score entries kept by the mask
 };
 
 __device__ __forceinline__ void report(DevStatus* st, int code, int where) {

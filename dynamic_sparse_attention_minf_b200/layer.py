@@ -62,9 +62,17 @@ def make_plan(w: Workload, device="cuda") -> LayerPlan:
     return plan
 
 
-def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None):
+# kernels launched per layer: VS estimation 6 (two score passes, row combine,
+# slash combine, two top-k), VS index build 3, BS estimation 3 (pool, pooled
+# scores, top-k), and one attention launch per pattern
+LAUNCHES_PER_STEP = 6 + 3 + 1 + 3 + 1 + 1
+
+
+def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None, marks=None):
     """Estimation, index build and sparse attention for every head of the
-    layer, in stream order; O (and LSE) are filled head by head."""
+    layer, in stream order; O (and LSE) are filled head by head.  ``marks``
+    (optional) gets ``mark(name)`` calls around the attention launches."""
+    mark = marks.mark if marks is not None else (lambda name: None)
     w, b = plan.w, plan.bufs
     shp = plan.shape
     L = minf.lib()
@@ -79,9 +87,11 @@ def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None):
         minf._check("minf_build_index", L.minf_build_index(
             minf.ctypes.byref(shp), nv, P(b["v_idx"]), w.k_v, P(b["s_idx"]), w.k_s, minf.ctypes.byref(ic),
             P(b["ws_vs_idx"]), b["ws_vs_idx"].numel(), st))
+        mark("vs_attn:pre")
         minf._check("minf_sparse_attn_vs", L.minf_sparse_attn_vs(
             minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.vs_heads), nv, minf.ctypes.byref(ic),
             w.k_v, w.k_s, P(o), P(lse), P(b["ws_vs_attn"]), b["ws_vs_attn"].numel(), st))
+        mark("vs_attn:post")
     if plan.bs_heads is not None:
         nbh = plan.bs_heads.numel()
         minf._check("minf_estimate_bs", L.minf_estimate_bs(

@@ -29,7 +29,10 @@
  *    minf_workspace_size(); its first 256 bytes hold a device status word
  *    that kernels set on a device-side error (a bounded wait that ran out,
  *    an index out of range).  Zero the workspace once before first use;
- *    read and clear the status with minf_get_device_status().
+ *    read and clear the status with minf_get_device_status().  The attention
+ *    calls also add two work counters there, as uint64 at byte offsets 8 and
+ *    16: the 128 x 128 key tiles they executed and the score entries their
+ *    masks kept (the useful entries); they are never reset by the library.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream) and returns a host-side status: launch errors
  *    come back as MINF_ERR_CUDA.

@@ -176,17 +176,18 @@ def bs_scores(qbar: np.ndarray, kbar: np.ndarray, scale: float) -> np.ndarray:
     return scale * (qbar @ kbar.T)
 
 
-def bs_select(q: np.ndarray, k: np.ndarray, scale: float, k_b: int, block: int = 64):
+def bs_select(q: np.ndarray, k: np.ndarray, scale: float, k_b: int, block: int = 64, blocks=None):
     """Per query block b, the k_b best key blocks c <= b by pooled score,
     with c = b forced.  No softmax: it is monotone within a row, so it cannot
     change the selection.  Returns idx [nb, k_b] (ascending, -1 padded) and
-    cnt [nb] = min(b + 1, k_b)."""
+    cnt [nb] = min(b + 1, k_b).  With ``blocks`` given, only those query
+    blocks are selected (rows of the result follow ``blocks``)."""
     qbar = bs_pool(q, block)
     kbar = bs_pool(k, block)
     nb = qbar.shape[0]
-    t = bs_scores(qbar, kbar, scale)
-    b = np.arange(nb)
-    valid = b[None, :] <= b[:, None]
+    b = np.arange(nb) if blocks is None else np.asarray(blocks, np.int64)
+    t = bs_scores(qbar[b], kbar, scale)
+    valid = np.arange(nb)[None, :] <= b[:, None]
     return select_topk_rows(t, valid, k_b, forced_col=b)
 
 
