@@ -256,3 +256,26 @@ def minf_dense_attn(q, k, v, heads=None, o=None, lse=None, want_lse=True, scale=
 
 def minf_get_device_status(ws, stream=None):
     return lib().minf_get_device_status(_p(ws), _stream(stream))
+
+
+def minf_estimate_vs_noalloc(q, k, heads, k_v, k_s, last_q=64, scale=0.0, return_scores=False, stream=None):
+    """minf_estimate_vs without a workspace: the library's built-in scratch
+    array is used, so this call allocates nothing on the device beyond the
+    outputs it is handed here (see include/minf.h for the limits)."""
+    L = lib()
+    fn = L.minf_estimate_vs_noalloc
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    shp = shape_of(q, k, scale)
+    hd = _heads(heads, q.device)
+    nh = hd.numel()
+    v_idx = torch.empty(shp.B, nh, k_v, dtype=torch.int32, device=q.device)
+    s_idx = torch.empty(shp.B, nh, k_s, dtype=torch.int32, device=q.device)
+    vs = ss = None
+    if return_scores:
+        vs = torch.empty(shp.B, nh, shp.N, dtype=torch.float32, device=q.device)
+        ss = torch.empty(shp.B, nh, shp.N, dtype=torch.float32, device=q.device)
+    _check("minf_estimate_vs_noalloc", fn(ctypes.byref(shp), _p(q), _p(k), _p(hd), nh, last_q, k_v, k_s,
+                                          _p(v_idx), _p(s_idx), _p(vs), _p(ss), _stream(stream)))
+    return (v_idx, s_idx, vs, ss) if return_scores else (v_idx, s_idx)

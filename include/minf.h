@@ -135,6 +135,27 @@ minf_status minf_estimate_vs(const minf_shape* shape, const minf_bf16* Q, const 
                              void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Allocation-free variant of minf_estimate_vs.  The paper has no counterpart:
+ * this exists for callers that cannot allocate device memory where they run
+ * the estimation (for example code inside a CUDA-graph capture that forbids
+ * allocation, or an engine plugin whose memory was planned up front), so they
+ * cannot provide a workspace.  Arguments and results are those of
+ * minf_estimate_vs without ws / ws_bytes; the scratch space is a 64 MiB array
+ * built into the library, held on every GPU that loads it until the process
+ * exits.  Problems that need more scratch than that (minf_workspace_size for
+ * MINF_OP_ESTIMATE_VS above 64 MiB, about 3.5M (batch x heads x tokens))
+ * are rejected with MINF_ERR_WORKSPACE_TOO_SMALL before anything runs.  The
+ * call allocates nothing.  Its first call on a device looks up the array's
+ * device address, so make that call before any stream capture begins.  All
+ * calls share the one array: calls that overlap on the GPU race, so
+ * serialise them.  This variant has no readable device status word.
+ */
+minf_status minf_estimate_vs_noalloc(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K,
+                                     const int32_t* heads, int nh, int last_q, int k_v, int k_s,
+                                     int32_t* v_idx, int32_t* s_idx, float* v_score, float* s_score,
+                                     void* stream);
+
+/*
  * Block-Sparse index estimation (summary, "Key points": queries and keys are
  * mean-pooled in 64-token blocks).  Pooled means are taken in fp32 and the
  * pooled scores t[b, c] = scale * Qbar_b . Kbar_c (c <= b) are formed with fp32

@@ -1,0 +1,77 @@
+"""The allocation-free Vertical-Slash estimation entry point.
+
+minf_estimate_vs_noalloc serves callers that cannot allocate device memory
+when they run the estimation (a graph capture that forbids allocation, an
+engine plugin with pre-planned memory), so they have no workspace to pass.
+It must give exactly what minf_estimate_vs gives with a workspace, call
+after call, although every call reuses the same built-in scratch array.
+This file is collected last so that a failure here never hides the others.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from dynamic_sparse_attention_minf_b200 import minf
+from dynamic_sparse_attention_minf_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    minf.lib()
+
+
+def _call_noalloc(q, k, heads, k_v, k_s):
+    """Through the C ABI directly (ctypes), with only inputs and outputs."""
+    L = minf.lib()
+    fn = L.minf_estimate_vs_noalloc
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(minf.Shape), vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    shp = minf.shape_of(q, k)
+    hd = torch.tensor(heads, dtype=torch.int32, device=q.device)
+    nh = len(heads)
+    v_idx = torch.full((1, nh, k_v), -7, dtype=torch.int32, device=q.device)
+    s_idx = torch.full((1, nh, k_s), -7, dtype=torch.int32, device=q.device)
+    vs = torch.full((1, nh, shp.N), -1.0, dtype=torch.float32, device=q.device)
+    ss = torch.full((1, nh, shp.N), -1.0, dtype=torch.float32, device=q.device)
+    code = fn(ctypes.byref(shp), ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+              ctypes.c_void_p(hd.data_ptr()), nh, 64, k_v, k_s, ctypes.c_void_p(v_idx.data_ptr()),
+              ctypes.c_void_p(s_idx.data_ptr()), ctypes.c_void_p(vs.data_ptr()), ctypes.c_void_p(ss.data_ptr()),
+              ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert code == 0, code
+    torch.cuda.synchronize()
+    return v_idx, s_idx, vs, ss
+
+
+def _reference(q, k, heads, k_v, k_s):
+    return minf.minf_estimate_vs(q, k, heads, k_v, k_s, return_scores=True)
+
+
+def test_noalloc_matches_workspace_entry_point_twice_in_a_row():
+    cases = [(wl.config(0), [0]),
+             (wl.small(Hq=4, Hkv=2, N=2048, d=128, seed=31, k_v=64, k_s=128), [3, 0, 2])]
+    for w, heads in cases:
+        q, k, _ = wl.make_qkv(w, "cuda")
+        ref = _reference(q, k, heads, w.k_v, w.k_s)
+        for _ in range(2):                       # second call sees the first call's leftovers
+            got = _call_noalloc(q, k, heads, w.k_v, w.k_s)
+            assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1])
+            np.testing.assert_allclose(got[2].cpu().numpy(), ref[2].cpu().numpy(), rtol=1e-4, atol=1e-7)
+            np.testing.assert_allclose(got[3].cpu().numpy(), ref[3].cpu().numpy(), rtol=1e-4, atol=1e-7)
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    L = minf.lib()
+    fn = L.minf_estimate_vs_noalloc
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(minf.Shape), vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    big = minf.Shape(1, 32, 8, 1048576, 128, 0.0)    # 32 heads x 1M tokens: far above 64 MiB
+    fake = ctypes.c_void_p(1 << 20)
+    assert fn(ctypes.byref(big), fake, fake, fake, 32, 64, 8, 8, fake, fake, None, None, None) == 4
