@@ -370,6 +370,33 @@ def run_ours(args, dist, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+def run_kernel_case(args):
+    """One kernel on a small case, for profilers: ``--kernel dense|vs`` at
+    ``--N`` tokens (8 query / 2 KV heads, d = 128; the VS case uses the 1M
+    workload's budgets, vertical 2000 / slash 12000).  The index is built
+    once; then the kernel runs ``--warmup`` + ``--steps`` times."""
+    from dynamic_sparse_attention_minf_b200 import layer, minf
+    from dynamic_sparse_attention_minf_b200 import workloads as wl
+    w = wl.config(WORKLOAD_ID, N=args.N)
+    w.Hq, w.Hkv = 8, 2
+    w.patterns = [wl.PAT_VS] * 8
+    q, k, v = wl.make_qkv(w, "cuda")
+    o = torch.empty_like(q)
+    if args.kernel == "vs":
+        plan = layer.make_plan(w, "cuda")
+        layer.run_layer(plan, q, k, v, o)
+        b = plan.bufs
+        fn = lambda: minf.minf_sparse_attn_vs(q, k, v, plan.vs_heads, b["vs_index"], o=o, want_lse=False,
+                                              ws=b["ws_vs_attn"])
+    else:
+        ws = minf.workspace(minf.OP_DENSE_ATTN, minf.shape_of(q, k), 1)
+        fn = lambda: minf.minf_dense_attn(q, k, v, [0], o=o, want_lse=False, ws=ws)
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel": args.kernel, "N": args.N, "launches": args.warmup + args.steps}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -378,7 +405,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense baseline")
+    ap.add_argument("--kernel", choices=["dense", "vs"], default=None,
+                    help="run only this attention kernel on a small case (for profiling)")
+    ap.add_argument("--N", type=int, default=262144, help="tokens of the --kernel case")
     args = ap.parse_args()
+    if args.kernel:
+        run_kernel_case(args)
+        return
     dist, rank, world, local = _dist()
     try:
         if args.impl == "reference":

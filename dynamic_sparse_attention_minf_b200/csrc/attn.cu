@@ -625,29 +625,31 @@ __global__ void __launch_bounds__(320, 1)
       if (kind == KIND_END) break;
       if (!warp_wait(&s_full[wg], n & 1, abort, p.status, 11)) break;
       tc_fence_after();
+      const int flags = dd.flags;
+      // Membership words of this warp's 64-row half, one per 32-column chunk.
+      // All rows of a warp lie in one half, so the chunk tests are warp-uniform:
+      // full chunks need no masking, empty chunks are not exponentiated.
+      uint32_t mw[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+      if (flags & F_MASK) {
+        const uint4 m4 = *reinterpret_cast<const uint4*>(&dd.mask[half][0]);
+        mw[0] = m4.x; mw[1] = m4.y; mw[2] = m4.z; mw[3] = m4.w;
+      }
       uint32_t sr[4][32];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(srow + wg * 128 + c4 * 32, sr[c4]);
+      for (int c4 = 0; c4 < 4; ++c4)
+        tmem_ld32(srow + wg * 128 + c4 * 32, sr[c4]);
       tmem_wait_ld();
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) reg_fence(sr[c4]);
       float s[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
-
-      const int flags = dd.flags;
-      if (!(flags & (F_CAUSAL | F_ASHAPE))) {
-        nnz += (flags & F_MASK) ? __popc(dd.mask[half][0]) + __popc(dd.mask[half][1]) +
-                                      __popc(dd.mask[half][2]) + __popc(dd.mask[half][3])
-                                : 128u;
-      }
-      if (flags & F_MASK) {
-        const uint32_t mw0 = dd.mask[half][0], mw1 = dd.mask[half][1];
-        const uint32_t mw2 = dd.mask[half][2], mw3 = dd.mask[half][3];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const uint32_t mw = (c < 32) ? mw0 : (c < 64) ? mw1 : (c < 96) ? mw2 : mw3;
-          if (!((mw >> (c & 31)) & 1u)) s[c] = -INFINITY;
+      for (int c4 = 0; c4 < 4; ++c4) {
+        if (mw[c4] != 0xFFFFFFFFu && mw[c4] != 0u) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (!((mw[c4] >> e) & 1u)) s[c4 * 32 + e] = -INFINITY;
         }
       }
       if (flags & (F_CAUSAL | F_ASHAPE)) {
@@ -669,14 +671,29 @@ __global__ void __launch_bounds__(320, 1)
             if (causal && j > i) s[c] = -INFINITY;
           }
         }
-      }
-      if (flags & (F_CAUSAL | F_ASHAPE)) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) nnz += (s[c] != -INFINITY);
-      }
-      float mx = -INFINITY;
+        for (int c4 = 0; c4 < 4; ++c4) {
+          if (mw[c4] != 0u) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            for (int e = 0; e < 32; ++e) nnz += (s[c4 * 32 + e] != -INFINITY);
+          }
+        }
+      } else {
+        nnz += __popc(mw[0]) + __popc(mw[1]) + __popc(mw[2]) + __popc(mw[3]);
+      }
+      // row max: eight independent chains over the non-empty chunks
+      float mx8[8];
+#pragma unroll
+      for (int k8 = 0; k8 < 8; ++k8) mx8[k8] = -INFINITY;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        if (mw[c4] != 0u) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[c4 * 32 + e]);
+        }
+      }
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_new = fmaxf(m_run, mx * sl2);
       float alpha = 1.f;
       const bool resc = m_new > m_run + 8.f;
@@ -685,8 +702,31 @@ __global__ void __launch_bounds__(320, 1)
         m_run = m_new;
       }
       const float msub = (m_run == -INFINITY) ? 0.f : m_run;
-      float lsum = 0.f;
-      // lazy correction of the running output (rare after the first tiles)
+      // P = 2^(s * scale * log2 e - m) as bf16 pairs over S's columns; a
+      // quarter of the exponentials run on the FMA pipe to relieve the MUFU.
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t pk[16];
+        if (mw[c4] != 0u) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float x0 = fmaf(s[c4 * 32 + e], sl2, -msub);
+            const float x1 = fmaf(s[c4 * 32 + e + 1], sl2, -msub);
+            const float p0 = fast_exp2(x0);
+            const float p1 = fast_exp2(x1);
+            ls4[(e >> 1) & 3] += p0 + p1;
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
+        }
+        tmem_st16(srow + wg * 128 + c4 * 16, pk);
+      }
+      l_run = l_run * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
+      // lazy correction of the running output (rare after the first tiles),
+      // done after the P stores so that the scores are no longer live
       if (__any_sync(0xFFFFFFFFu, resc && n > 0)) {
         if (!warp_wait(&o_done[wg], (n - 1) & 1, abort, p.status, 12)) break;
         tc_fence_after();
@@ -702,20 +742,6 @@ __global__ void __launch_bounds__(320, 1)
           tmem_st32(orow + c0, o);
         }
       }
-      // P = exp2(s * scale * log2 e - m), written as bf16 pairs over S's columns
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = fast_exp2(fmaf(s[c4 * 32 + e], sl2, -msub));
-          const float p1 = fast_exp2(fmaf(s[c4 * 32 + e + 1], sl2, -msub));
-          lsum += p0 + p1;
-          pk[e >> 1] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(srow + wg * 128 + c4 * 16, pk);
-      }
-      l_run = l_run * alpha + lsum;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[wg]);

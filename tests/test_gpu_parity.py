@@ -81,9 +81,12 @@ def _vs_pipeline(w, heads, rows=None):
         ov, os_ = orc.vs_select(rv, rs, w.k_v, w.k_s)
         check_index_set(gv[hi], ov, rv, what=f"vertical h{h}")
         check_index_set(gs[hi], os_, rs, forced=0, what=f"slash h{h}")
-    index = minf.minf_build_index(minf.shape_of(q, k), v_idx, s_idx)
-    o, lse = minf.minf_sparse_attn_vs(q, k, v, heads, index)
-    torch.cuda.synchronize()
+    ws_i = minf.workspace(minf.OP_BUILD_INDEX, minf.shape_of(q, k), len(heads))
+    index = minf.minf_build_index(minf.shape_of(q, k), v_idx, s_idx, ws=ws_i)
+    ws_a = minf.workspace(minf.OP_SPARSE_ATTN_VS, minf.shape_of(q, k), len(heads))
+    o, lse = minf.minf_sparse_attn_vs(q, k, v, heads, index, ws=ws_a)
+    assert minf.minf_get_device_status(ws_i) == 0
+    assert minf.minf_get_device_status(ws_a) == 0
     # index build is integer work: bit-exact against the oracle on the GPU's own V and S
     for hi in range(len(heads)):
         groups, vcnt, vidx = orc.vs_build_index(gv[hi], gs[hi], w.N)
@@ -137,7 +140,9 @@ def test_vs_index_from_oracle_sets():
     v_idx = torch.tensor(np.stack([V, V])[None], dtype=torch.int32, device=DEV)
     s_idx = torch.tensor(np.stack([S, S])[None], dtype=torch.int32, device=DEV)
     index = minf.minf_build_index(minf.shape_of(q, k), v_idx, s_idx)
-    o, lse = minf.minf_sparse_attn_vs(q, k, v, [0, 1], index)
+    ws_a = minf.workspace(minf.OP_SPARSE_ATTN_VS, minf.shape_of(q, k), 2)
+    o, lse = minf.minf_sparse_attn_vs(q, k, v, [0, 1], index, ws=ws_a)
+    assert minf.minf_get_device_status(ws_a) == 0
     _check_attn(o, lse, qn, kn, vn, [0, 1], w, lambda hi, h: (lambda r: orc.mask_vs(r, w.N, V, S)))
 
 
@@ -163,8 +168,9 @@ def _bs_pipeline(w, heads, rows=None):
             flips += check_index_set(gi[hi, b, :gc[hi, b]], ri[b, :rc[b]], tref[b, :b + 1], forced=b,
                                      what=f"h{h} block {b}")
             assert (gi[hi, b, gc[hi, b]:] == -1).all()
-    o, lse = minf.minf_sparse_attn_bs(q, k, v, heads, blk_idx, blk_cnt)
-    torch.cuda.synchronize()
+    ws_a = minf.workspace(minf.OP_SPARSE_ATTN_BS, minf.shape_of(q, k), len(heads))
+    o, lse = minf.minf_sparse_attn_bs(q, k, v, heads, blk_idx, blk_cnt, ws=ws_a)
+    assert minf.minf_get_device_status(ws_a) == 0
     _check_attn(o, lse, qn, kn, vn, heads, w,
                 lambda hi, h: (lambda r: orc.mask_bs(r, w.N, gi[hi], gc[hi])), rows)
     return flips
