@@ -548,9 +548,14 @@ __global__ void __launch_bounds__(320, 1)
       for (int h = 0; h < D / 64; ++h) tma_load_2d(smem + C::kOffQ + h * C::kRegion, &tmQ, q_full, 64 * h, qrow);
     }
     __syncwarp();
-    produce_tiles<D, POL>(P, p, b, hi, qt);
-    if (lane == 0 && P.ok) atomicAdd(&p.status->tiles, (unsigned long long)P.t);
-    P.emit_end();
+    // Failure-detection test hook: the first CTA withholds every key tile,
+    // so its consumers' bounded waits run out and the call reports a timeout.
+    const bool withhold = p.status->withhold != 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+    if (!withhold) {
+      produce_tiles<D, POL>(P, p, b, hi, qt);
+      if (lane == 0 && P.ok) atomicAdd(&p.status->tiles, (unsigned long long)P.t);
+      P.emit_end();
+    }
     P.flush_pending();
     P.drain();
     if (lane == 0) {

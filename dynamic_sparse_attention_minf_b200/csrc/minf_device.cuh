@@ -22,6 +22,7 @@ struct DevStatus {
   int where;
   unsigned long long tiles;  // attention: 128 x 128 key tiles executed
   unsigned long long nnz;    // attention: score entries kept by the mask
+  int withhold;              // test hook: attention CTA (0,0,0) issues no key tiles
 };
 
 __device__ __forceinline__ void report(DevStatus* st, int code, int where) {

@@ -33,6 +33,11 @@
  *    calls also add two work counters there, as uint64 at byte offsets 8 and
  *    16: the 128 x 128 key tiles they executed and the score entries their
  *    masks kept (the useful entries); they are never reset by the library.
+ *    The int32 at byte offset 24 is a failure-detection test hook: while it
+ *    is non-zero, the first CTA of every attention call withholds its key
+ *    tiles, its bounded waits (2 s) run out, and the call's status becomes
+ *    MINF_ERR_DEVICE_TIMEOUT without faulting or hanging the GPU.  Keep it
+ *    zero in normal use.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream) and returns a host-side status: launch errors
  *    come back as MINF_ERR_CUDA.
