@@ -336,21 +336,54 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi
     const int* tg = p.tgrp + hrow * p.k_s * 2;
     const int G = p.tgrp_cnt[hrow];
     const uint32_t* W = p.wmap + hrow * p.wmap_words;
-    // slash bands: ascending keys = descending offsets
-    for (int g = G - 1; g >= 0 && P.ok; --g) {
-      const int A = tg[2 * g], Bo = tg[2 * g + 1];
-      const int hi_key = min(R + 127 - A, p.N - 1);
-      if (hi_key < 0) continue;
-      const int lo_key = max(0, R - Bo);
-      for (int j0 = lo_key; j0 <= hi_key && P.ok; j0 += 128) {
-        const int cnt = min(128, hi_key - j0 + 1);
+    // Slash bands, in ascending keys = descending offsets.  Only tile groups
+    // with a_G <= R + 127 reach this query tile: binary-search the last one,
+    // then walk down 32 groups at a time, one group per lane, each lane
+    // fetching its group's first-tile mask words so that the loads of a batch
+    // overlap instead of costing a round trip per group.
+    int top = 0;
+    {
+      int lo = 0, hi2 = G;
+      while (lo < hi2) {
+        const int mid = (lo + hi2) >> 1;
+        if (__ldg(tg + 2 * mid) <= R + 127) lo = mid + 1; else hi2 = mid;
+      }
+      top = lo - 1;
+    }
+    auto tile_word = [&](int j0, int cnt, int hh, int wd) -> uint32_t {
+      const int x0 = R + 64 * hh - j0 + 63 - 32 * wd;
+      return __brev(wmap_window(W, x0 - 31)) & count_mask(cnt, wd);
+    };
+    for (int base = top; base >= 0 && P.ok; base -= 32) {
+      const int gl = base - lane;
+      int lo_l = 0, hi_l = -1;
+      uint32_t w8[8];
+      if (gl >= 0) {
+        const int A = __ldg(tg + 2 * gl), Bo = __ldg(tg + 2 * gl + 1);
+        hi_l = min(R + 127 - A, p.N - 1);
+        lo_l = max(0, R - Bo);
+        const int cnt = min(128, hi_l - lo_l + 1);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) w8[q] = tile_word(lo_l, cnt, q >> 2, q & 3);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) w8[q] = 0u;
+      }
+      const int nbatch = min(32, base + 1);
+      for (int k = 0; k < nbatch && P.ok; ++k) {
+        const int lo_key = __shfl_sync(0xFFFFFFFFu, lo_l, k);
+        const int hi_key = __shfl_sync(0xFFFFFFFFu, hi_l, k);
         uint32_t word = 0xFFFFFFFFu;
-        if (lane < 8) {
-          const int hh = lane >> 2, wd = lane & 3;
-          const int x0 = R + 64 * hh - j0 + 63 - 32 * wd;
-          word = __brev(wmap_window(W, x0 - 31)) & count_mask(cnt, wd);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t v = __shfl_sync(0xFFFFFFFFu, w8[q], k);
+          if (lane == q) word = v;
         }
-        P.emit_range(j0, j0 + 64, word, (j0 + cnt - 1 > R) ? F_CAUSAL : 0);
+        for (int j0 = lo_key; j0 <= hi_key && P.ok; j0 += 128) {
+          const int cnt = min(128, hi_key - j0 + 1);
+          if (j0 != lo_key && lane < 8) word = tile_word(j0, cnt, lane >> 2, lane & 3);
+          P.emit_range(j0, j0 + 64, word, (j0 + cnt - 1 > R) ? F_CAUSAL : 0);
+        }
       }
     }
     // verticals: V_{b1} (both halves as applicable), then V_{b0} on half-1 bands
@@ -589,7 +622,9 @@ __global__ void __launch_bounds__(320, 1)
         const int st = t % C::kStages;
         if (!mbar_wait(&k_full[st], (t / C::kStages) & 1, abort, p.status, 5)) { ok = false; break; }
         if (desc[st].kind == KIND_END) break;
-        tc_fence_after();
+        // Q and K were written by TMA or by cp.async plus the producer's proxy
+        // fence; the barrier alone orders them before the MMA (no tcgen05
+        // fence here: it would stall the issue of every tile).
         const int w = t & 1;
         const uint32_t kaddr = smem_u32(smem + C::kOffK + st * C::kKVBytes);
 #pragma unroll
