@@ -742,20 +742,21 @@ __global__ void __launch_bounds__(320, 1)
         m_run = m_new;
       }
       const float msub = (m_run == -INFINITY) ? 0.f : m_run;
-      // P = 2^(s * scale * log2 e - m) as bf16 pairs over S's columns; a
-      // quarter of the exponentials run on the FMA pipe to relieve the MUFU.
-      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      // P = 2^(s * scale * log2 e - m) as bf16 pairs over S's columns; the
+      // argument and the row sum use packed two-lane fp32 instructions.
+      const uint64_t sl2x2 = f32x2_pack(sl2, sl2), nm2 = f32x2_pack(-msub, -msub);
+      uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t pk[16];
         if (mw[c4] != 0u) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float x0 = fmaf(s[c4 * 32 + e], sl2, -msub);
-            const float x1 = fmaf(s[c4 * 32 + e + 1], sl2, -msub);
+            float x0, x1;
+            f32x2_unpack(f32x2_fma(f32x2_pack(s[c4 * 32 + e], s[c4 * 32 + e + 1]), sl2x2, nm2), x0, x1);
             const float p0 = fast_exp2(x0);
             const float p1 = fast_exp2(x1);
-            ls4[(e >> 1) & 3] += p0 + p1;
+            acc2[(e >> 1) & 1] = f32x2_add(acc2[(e >> 1) & 1], f32x2_pack(p0, p1));
             pk[e >> 1] = pack_bf16x2(p0, p1);
           }
         } else {
@@ -764,7 +765,10 @@ __global__ void __launch_bounds__(320, 1)
         }
         tmem_st16(srow + wg * 128 + c4 * 16, pk);
       }
-      l_run = l_run * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
+      float a0, a1, b0, b1;
+      f32x2_unpack(acc2[0], a0, a1);
+      f32x2_unpack(acc2[1], b0, b1);
+      l_run = l_run * alpha + ((a0 + a1) + (b0 + b1));
       // lazy correction of the running output (rare after the first tiles),
       // done after the P stores so that the scores are no longer live
       if (__any_sync(0xFFFFFFFFu, resc && n > 0)) {
