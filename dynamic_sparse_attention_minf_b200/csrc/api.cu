@@ -209,7 +209,12 @@ minf_status minf_estimate_vs(const minf_shape* s, const minf_bf16* Q, const minf
   p.dpart = w.dpart;
   p.status = w.status;
   cudaStream_t cs = (cudaStream_t)stream;
-  cudaError_t e = vs_estimate_launch(p, cs);
+  CUtensorMap tq, tk;
+  if (((uintptr_t)Q | (uintptr_t)K) & 15) return MINF_ERR_INVALID_ARG;
+  if (!make_map(&tq, Q, (long long)s->B * s->Hq * s->N, s->d, 128) ||
+      !make_map(&tk, K, (long long)s->B * s->Hkv * s->N, s->d, 64))
+    return MINF_ERR_CUDA;
+  cudaError_t e = vs_estimate_tc_launch(tq, tk, p, cs);
   if (e != cudaSuccess) return MINF_ERR_CUDA;
   TopkRows t;
   t.scores = p.v_score;

@@ -214,6 +214,17 @@ __global__ void __launch_bounds__(256) vs_slash_kernel(const VsEstParams p, int 
   p.s_score[bh * p.N + o] = s;
 }
 
+cudaError_t vs_combine_launch(const VsEstParams& p, int nparts, cudaStream_t stream) {
+  vs_combine_kernel<<<dim3(64, p.nh, p.B), 256, 0, stream>>>(p, nparts);
+  return cudaGetLastError();
+}
+
+cudaError_t vs_slash_launch(const VsEstParams& p, cudaStream_t stream) {
+  const int ntiles = (p.N + kVsKeys - 1) / kVsKeys;
+  vs_slash_kernel<<<dim3((p.N + 255) / 256, p.nh, p.B), 256, 0, stream>>>(p, ntiles);
+  return cudaGetLastError();
+}
+
 cudaError_t vs_estimate_launch(const VsEstParams& p, cudaStream_t stream) {
   const int ntiles = (p.N + kVsKeys - 1) / kVsKeys;
   dim3 grid(ntiles, p.nh, p.B);

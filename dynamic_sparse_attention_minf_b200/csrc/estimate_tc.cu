@@ -1,0 +1,287 @@
+// Vertical-Slash index estimation on the tensor cores ("MInference 1.0"
+// summary, "Key points": the last query vectors are scored against all keys).
+//
+// One CTA takes one head and a run of 128-key tiles.  The scores of the last
+// query rows against a key tile, S = Q_last K^T, are one tcgen05 GEMM (bf16
+// inputs, exact products, fp32 accumulation in TMEM).  Q's last 128 rows are
+// the A operand; the real rows are the last `last_q` <= 64 of them, in TMEM
+// lanes 64..127, read by warps 2, 3, 6, 7 (two threads per row, 64 columns
+// each).  K tiles stream through a 3-stage TMA ring.
+//
+//  pass 1: each thread keeps an online (max, sum) of 2^(s * scale * log2 e)
+//          over its columns of the CTA's tiles; the two halves of a row are
+//          merged and written as the CTA's partial of that row.
+//  pass 2: p = 2^(x - m) / l with the combined row statistics is written to
+//          shared memory, and 128 threads form, in a fixed order, the column
+//          sums (vertical scores) and the tile's 191 diagonal partials.
+//
+// warp 0 lane 0: TMA producer; warp 1: TMEM owner and MMA issuer;
+// warps 2, 3, 6, 7: score warps; warps 4, 5 idle.
+#include <algorithm>
+
+#include "minf_device.cuh"
+#include "minf_internal.h"
+
+namespace minf {
+
+template <int D>
+struct EstCfg {
+  static constexpr int kThreads = 256;
+  static constexpr int kRegion = 128 * 128;
+  static constexpr int kTileBytes = 128 * D * 2;  // 128 rows (Q) or 128 keys (K)
+  static constexpr int kStages = 3;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kTileBytes;
+  static constexpr int kOffP = kOffK + kStages * kTileBytes;  // pass 2: 2 x [64][129] fp32
+  static constexpr int kPStride = 129;
+  static constexpr int kPBytes = 64 * kPStride * 4;
+  static constexpr int kOffBars = kOffP + 2 * kPBytes;
+  // barriers: q_full, k_full[3], k_empty[3], s_full[2], s_free[2], mma_done
+  static constexpr int kNumBars = 1 + 2 * kStages + 4 + 1;
+  static constexpr int kOffMisc = kOffBars + kNumBars * 8;
+  static constexpr int kOffXch = kOffMisc + 16;             // pass 1: [2][64][2] fp32
+  static constexpr int kSmem = kOffXch + 2 * 64 * 2 * 4;
+  static_assert(kSmem <= 232448, "shared memory budget");
+  static constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);
+};
+
+template <int D, int PASS>
+__global__ void __launch_bounds__(256, 1)
+    vs_est_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const VsEstParams p, int tiles_per_cta, int nchunks) {
+  using C = EstCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
+  const int head = p.heads[hi];
+  if ((smem_u32(smem) & 1023u) != 0u || head < 0 || head >= p.Hq) {
+    if (threadIdx.x == 0) report(p.status, MINF_ERR_DEVICE_BOUNDS, 60);
+    return;
+  }
+  const int kvh = head / p.group;
+  const int ntiles = (p.N + 127) / 128;
+  const int t0 = chunk * tiles_per_cta;
+  const int nt = min(ntiles, t0 + tiles_per_cta) - t0;
+  const size_t bh = (size_t)b * p.nh + hi;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + C::kStages;
+  uint64_t* s_full = k_empty + C::kStages;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* mma_done = s_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&s_free[w], 128);
+    }
+    mbar_init(mma_done, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, C::kTileBytes);
+      const int qrow0 = (b * p.Hq + head) * p.N + p.N - 128;
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) tma_load_2d(smem + C::kOffQ + h * C::kRegion, &tmQ, q_full, 64 * h, qrow0);
+      const int kv_row0 = (b * p.Hkv + kvh) * p.N;
+      int issued = 0;
+      for (int k = 0; k < nt; ++k) {
+        const int st = k % C::kStages;
+        if (k >= C::kStages && !mbar_wait(&k_empty[st], ((k / C::kStages) - 1) & 1, abort, p.status, 61)) break;
+        const int j0 = (t0 + k) * 128;
+        uint8_t* kb = smem + C::kOffK + st * C::kTileBytes;
+        mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_2d(kb + h * C::kRegion, &tmK, &k_full[st], 64 * h, kv_row0 + j0);
+          tma_load_2d(kb + h * C::kRegion + 8192, &tmK, &k_full[st], 64 * h, kv_row0 + j0 + 64);
+        }
+        issued = k + 1;
+      }
+      int dummy = 0;  // never exit with copies in flight
+      for (int k = max(0, issued - C::kStages); k < issued; ++k)
+        mbar_wait(&k_full[k % C::kStages], (k / C::kStages) & 1, &dummy, p.status, 62);
+      mbar_wait(q_full, 0, &dummy, p.status, 63);
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(q_full, 0, abort, p.status, 64);
+      const uint32_t qaddr = smem_u32(smem + C::kOffQ);
+      for (int k = 0; k < nt && ok; ++k) {
+        const int st = k % C::kStages, buf = k & 1;
+        ok = mbar_wait(&k_full[st], (k / C::kStages) & 1, abort, p.status, 65);
+        if (ok && k >= 2) ok = mbar_wait(&s_free[buf], ((k >> 1) - 1) & 1, abort, p.status, 66);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(smem + C::kOffK + st * C::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kRegion + (kk & 3) * 32;
+          umma_ss(tmem + buf * 128, sdesc_sw128(qaddr + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024),
+                  C::kIdescS, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[buf]);
+        umma_commit(&k_empty[st]);
+      }
+      umma_commit(mma_done);
+      int dummy = 0;
+      mbar_wait(mma_done, 0, &dummy, p.status, 67);
+    }
+    __syncwarp();
+  } else if ((warp & 3) >= 2) {
+    // ------------------------------------------------------- score warps
+    const int qq = warp & 3;          // TMEM lane quarter 2 or 3: rows 64..127 of the Q tile
+    const int hc = warp >> 2;         // key columns 64 hc .. 64 hc + 63 of every tile
+    const int r = qq * 32 + lane;
+    const int qrow = r - 64;          // query row N - 64 + qrow
+    const int i = p.N - 128 + r;
+    const bool real = r >= 128 - p.last_q;
+    const int ctid = (hc * 2 + (qq - 2)) * 32 + lane;
+    const uint32_t taddr = tmem + ((uint32_t)(qq * 32) << 16) + hc * 64;
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    float mr = 0.f, il = 0.f;
+    if (PASS == 2 && real) {
+      mr = p.row_ml[(bh * 64 + qrow) * 2];
+      il = p.row_ml[(bh * 64 + qrow) * 2 + 1];
+    }
+    for (int k = 0; k < nt; ++k) {
+      const int buf = k & 1;
+      // all four score warps agree before going on (pass 2 meets at a
+      // barrier below, which a warp that gave up would never reach)
+      const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (k >> 1) & 1, abort, p.status, 68));
+      if (!bar_and(2, 128, got)) break;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      tmem_ld32(taddr + buf * 128, v0);
+      tmem_ld32(taddr + buf * 128 + 32, v1);
+      tmem_wait_ld();
+      reg_fence(v0);
+      reg_fence(v1);
+      tc_fence_before();
+      mbar_arrive(&s_free[buf]);
+      const int j0 = (t0 + k) * 128 + hc * 64;
+      float x[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float sv = __uint_as_float(c < 32 ? v0[c] : v1[c - 32]);
+        x[c] = (real && j0 + c <= i) ? sv * sl2 : -INFINITY;
+      }
+      if (PASS == 1) {
+        float m8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], x[c]);
+        const float tm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        if (tm > m) {
+          if (m != -INFINITY) l *= exp2f(m - tm);
+          m = tm;
+        }
+        if (m != -INFINITY) {
+          float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c = 0; c < 64; ++c) a4[c & 3] += exp2f(x[c] - m);
+          l += (a4[0] + a4[1]) + (a4[2] + a4[3]);
+        }
+      } else {
+        float* P = reinterpret_cast<float*>(smem + C::kOffP + buf * C::kPBytes);
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          P[qrow * C::kPStride + hc * 64 + c] = (x[c] == -INFINITY) ? 0.f : exp2f(x[c] - mr) * il;
+        named_bar_sync(1, 128);
+        const int jj = (t0 + k) * 128 + ctid;
+        float cs = 0.f;
+        for (int q = 0; q < 64; ++q) cs += P[q * C::kPStride + ctid];
+        if (jj < p.N) p.v_score[bh * p.N + jj] = cs;
+        for (int kd = ctid; kd < 191; kd += 128) {
+          float dsum = 0.f;
+          const int qlo = max(0, kd - 127), qhi = min(63, kd);
+          for (int q = qlo; q <= qhi; ++q) dsum += P[q * C::kPStride + (q - kd + 127)];
+          p.dpart[(bh * ntiles + t0 + k) * 192 + kd] = dsum;
+        }
+      }
+    }
+    if (PASS == 1) {
+      float* xch = reinterpret_cast<float*>(smem + C::kOffXch);
+      xch[(hc * 64 + qrow) * 2] = m;
+      xch[(hc * 64 + qrow) * 2 + 1] = l;
+      named_bar_sync(1, 128);
+      if (hc == 0) {
+        const float m1 = xch[(64 + qrow) * 2], l1 = xch[(64 + qrow) * 2 + 1];
+        const float M = fmaxf(m, m1);
+        float L = 0.f;
+        if (M != -INFINITY) {
+          if (m != -INFINITY) L += l * exp2f(m - M);
+          if (m1 != -INFINITY) L += l1 * exp2f(m1 - M);
+        }
+        float* out = p.part_ml + ((bh * nchunks + chunk) * 64 + qrow) * 2;
+        out[0] = M;
+        out[1] = L;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int D>
+static cudaError_t launch_est_tc(const CUtensorMap& tq, const CUtensorMap& tk, const VsEstParams& p,
+                                 cudaStream_t stream) {
+  using C = EstCfg<D>;
+  const int ntiles = (p.N + 127) / 128;
+  // about four CTAs per SM in all, at most 32 key tiles each
+  const long long units = (long long)ntiles * p.nh * p.B;
+  const int tpc = (int)std::max<long long>(1, std::min<long long>(32, (units + 591) / 592));
+  const int nchunks = (ntiles + tpc - 1) / tpc;
+  cudaError_t e = cudaFuncSetAttribute(vs_est_tc_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(vs_est_tc_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(nchunks, p.nh, p.B);
+  vs_est_tc_kernel<D, 1><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, p, tpc, nchunks);
+  e = vs_combine_launch(p, nchunks, stream);
+  if (e != cudaSuccess) return e;
+  vs_est_tc_kernel<D, 2><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, p, tpc, nchunks);
+  // the tile's score rows are the last 64 query rows (rows beyond last_q are
+  // zero), so the diagonal partials use the 64-row geometry
+  VsEstParams q64 = p;
+  q64.last_q = 64;
+  return vs_slash_launch(q64, stream);
+}
+
+cudaError_t vs_estimate_tc_launch(const CUtensorMap& tq, const CUtensorMap& tk, const VsEstParams& p,
+                                  cudaStream_t stream) {
+  if (p.d == 128) return launch_est_tc<128>(tq, tk, p, stream);
+  if (p.d == 64) return launch_est_tc<64>(tq, tk, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace minf
