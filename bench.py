@@ -287,11 +287,13 @@ def run_ours(args, dist, rank, world, local):
     per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     step_ms = ev[0].elapsed_time(ev[-1]) / args.steps
     step_ms = _max_over_ranks(dist, step_ms)
-    vs_ms = []
+    phases = {}
     for a, b in zip(marks[0::2], marks[1::2]):
-        if a[0] == "vs_attn:pre" and b[0] == "vs_attn:post":
-            vs_ms.append(a[1].elapsed_time(b[1]))
-    vs_ms = statistics.mean(vs_ms) if vs_ms else None
+        name = a[0].split(":")[0]
+        assert a[0] == name + ":pre" and b[0] == name + ":post"
+        phases.setdefault(name, []).append(a[1].elapsed_time(b[1]))
+    phase_ms = {n: round(statistics.mean(t), 3) for n, t in phases.items()}
+    vs_ms = phase_ms.get("vs_attn")
 
     # end to end through the public API: pinned host in, host out
     hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
@@ -359,6 +361,7 @@ def run_ours(args, dist, rank, world, local):
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs 12 GiB per step, larger than the 126 MB L2 (no flush needed)"},
         "step_ms_each": [round(x, 2) for x in per_step],
+        "phase_ms": phase_ms,
         "useful_tflop_per_step": useful / 1e12, "executed_tflop_per_step": executed / 1e12,
         "density_vs_dense": useful / dense_flops,
         "dense_attn_ms_est": dense_ms,

@@ -143,12 +143,13 @@ minf_status attn_common(int pol, const minf_shape* s, const minf_bf16* Q, const 
 }
 
 minf_status attn_launch(int pol, const minf_shape* s, const AttnParams& p, void* stream) {
-  CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, p.Q, (long long)s->B * s->Hq * s->N, s->d, 128) ||
-      !make_map(&tk, p.K, (long long)s->B * s->Hkv * s->N, s->d, 64) ||
-      !make_map(&tv, p.V, (long long)s->B * s->Hkv * s->N, s->d, 64))
+  CUtensorMap tq, tk, tv, tk2, tv2;
+  const long long kv_rows = (long long)s->B * s->Hkv * s->N;
+  if (!make_map(&tq, p.Q, (long long)s->B * s->Hq * s->N, s->d, 128) || !make_map(&tk, p.K, kv_rows, s->d, 64) ||
+      !make_map(&tv, p.V, kv_rows, s->d, 64) || !make_map(&tk2, p.K, kv_rows, s->d, 128) ||
+      !make_map(&tv2, p.V, kv_rows, s->d, 128))
     return MINF_ERR_CUDA;
-  return cuda_status(attn_dispatch(s->d, pol, tq, tk, tv, p, (cudaStream_t)stream));
+  return cuda_status(attn_dispatch(s->d, pol, tq, tk, tv, tk2, tv2, p, (cudaStream_t)stream));
 }
 
 }  // namespace

@@ -1,8 +1,8 @@
 // Causal (sparse) attention mainloop for sm_100a: one CTA per (batch, head,
 // 128-row query tile), warp-specialized.
 //
-//   warps 0-3  softmax warpgroup 0: key tiles 0, 2, 4, ...   (thread = query row)
-//   warps 4-7  softmax warpgroup 1: key tiles 1, 3, 5, ...
+//   warps 0-3  softmax warpgroup 0: key columns 0-63 of every tile  (thread = query row)
+//   warps 4-7  softmax warpgroup 1: key columns 64-127 of every tile
 //   warp  8    tcgen05 issuer (one lane) and TMEM owner
 //   warp  9    producer: enumerates the key tiles of the query tile for the
 //              head's pattern, writes each tile's descriptor (column ids and
@@ -10,12 +10,14 @@
 //              memory by TMA (contiguous 64-key chunks) or cp.async (gathered
 //              columns).
 //
-// Per key tile t (128 keys) the issuer computes S = Q K^T into the TMEM
-// buffer of warpgroup t&1; that warpgroup masks and exponentiates S, writes
-// P (bf16) back over S in TMEM and the issuer accumulates O_{t&1} += P V with
-// P read from TMEM.  The two warpgroups keep separate running max / sum and
-// separate O accumulators, merged in the epilogue, so that one warpgroup's
-// exponentials overlap the other's matrix products.
+// Per key tile t (128 keys) the issuer computes S = Q K^T into TMEM buffer
+// t&1.  Warpgroup w masks and exponentiates its 64 columns of S and writes P
+// (bf16) back over them in TMEM; the issuer then accumulates
+// O_w += P[:, 64w:64w+64] V[64w:64w+64, :] with P read from TMEM.  Each
+// warpgroup keeps its own running max / sum and O accumulator over its column
+// half of every tile, and the two are merged in the epilogue, so both
+// warpgroups work on every tile with no exchange between them, while the
+// issuer computes the next tile's scores into the other buffer.
 //
 // The four key sources ("MInference 1.0" summary, "Summary": A-shape,
 // Vertical-Slash, Block-Sparse; and dense causal attention as the baseline):
@@ -55,8 +57,9 @@ struct AttnCfg {
   static constexpr int kOffSCols = kOffDesc + kStages * (int)sizeof(TileDesc);
   static constexpr int kOffSBits = kOffSCols + 160 * 4;
   static constexpr int kOffBars = kOffSBits + 160;
-  // barriers: k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], q_full, mma_done
-  static constexpr int kNumBars = 3 * kStages + 8;
+  // barriers: k_full[S], v_full[S], k_empty[S], v_empty[S], d_empty[S], s_full[2], p_full[2],
+  // q_full, mma_done
+  static constexpr int kNumBars = 5 * kStages + 6;
   static constexpr int kOffMisc = kOffBars + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16;
   static_assert(kSmem <= 232448, "shared memory budget");
@@ -102,18 +105,23 @@ struct Producer {
   uint8_t* sbits;
   uint64_t* k_full;
   uint64_t* v_full;
-  uint64_t* kv_empty;
-  const CUtensorMap* tmK;
+  uint64_t* k_empty;
+  uint64_t* v_empty;
+  uint64_t* d_empty;
+  const CUtensorMap* tmK;   // 64-row boxes
   const CUtensorMap* tmV;
+  const CUtensorMap* tmK2;  // 128-row boxes, for two adjacent chunks
+  const CUtensorMap* tmV2;
   const __nv_bfloat16* Kh;  // this (batch, kv head)'s K rows
   const __nv_bfloat16* Vh;
   int kv_row0;
   int R;
   int N;
   int lane;
-  int t;
+  int t;        // tiles whose K side (and descriptor) has been emitted
+  int tv;       // tiles whose V side has been emitted: t - 1 (a range tile's V lags) or t
+  int vj0[2];   // key chunks of tile tv while its V lags
   int pending;  // stage whose gathered copies are issued but not yet signalled
-  int issued[C::kStages];
   volatile int* abort;
   DevStatus* st;
   bool ok;
@@ -131,12 +139,14 @@ struct Producer {
     }
   }
 
-  // Claims the stage of tile t; false on abort.
-  __device__ bool acquire(int& stage) {
+  // Claims the K slot and the descriptor of tile t: S = Q K^T of tile t - S
+  // is done and the softmax warps have read its descriptor.  False on abort.
+  __device__ bool acquire_k(int& stage) {
     stage = t % C::kStages;
     if (t >= C::kStages) {
       flush_pending();
-      if (!warp_wait(&kv_empty[stage], ((t / C::kStages) - 1) & 1, abort, st, 1)) {
+      const uint32_t par = ((t / C::kStages) - 1) & 1;
+      if (!warp_wait(&k_empty[stage], par, abort, st, 1) || !warp_wait(&d_empty[stage], par, abort, st, 14)) {
         ok = false;
         return false;
       }
@@ -144,12 +154,48 @@ struct Producer {
     return true;
   }
 
+  // Claims the V slot of tile u: P V of tile u - S is done.
+  __device__ bool acquire_v(int u, int& stage) {
+    stage = u % C::kStages;
+    if (u >= C::kStages) {
+      flush_pending();
+      if (!warp_wait(&v_empty[stage], ((u / C::kStages) - 1) & 1, abort, st, 15)) {
+        ok = false;
+        return false;
+      }
+    }
+    return true;
+  }
+
+  // Issues the V loads of the range tile whose V lags behind its K.
+  __device__ void emit_v_lag() {
+    if (!ok || tv == t) return;
+    int stage;
+    if (!acquire_v(tv, stage)) return;
+    if (lane == 0) {
+      uint8_t* vb = smem + C::kOffV + stage * C::kKVBytes;
+      mbar_arrive_expect_tx(&v_full[stage], C::kKVBytes);
+      if (vj0[1] == vj0[0] + 64) {
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) tma_load_2d(vb + h * C::kRegion, tmV2, &v_full[stage], 64 * h, kv_row0 + vj0[0]);
+      } else {
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_2d(vb + h * C::kRegion, tmV, &v_full[stage], 64 * h, kv_row0 + vj0[0]);
+          tma_load_2d(vb + h * C::kRegion + 8192, tmV, &v_full[stage], 64 * h, kv_row0 + vj0[1]);
+        }
+      }
+    }
+    ++tv;
+  }
+
   // A tile of two 64-key chunks at keys j0a, j0b with per-half mask words
-  // (lane l < 8 holds word (l >> 2, l & 3)).
+  // (lane l < 8 holds word (l >> 2, l & 3)).  K is loaded now; V after the
+  // next tile's K, so that K loads run ahead of the V slots' release.
   __device__ void emit_range(int j0a, int j0b, uint32_t word, int flags) {
     if (!ok) return;
     int stage;
-    if (!acquire(stage)) return;
+    if (!acquire_k(stage)) return;
     TileDesc& dd = desc[stage];
     const bool full = __all_sync(0xFFFFFFFFu, lane >= 8 || word == 0xFFFFFFFFu);
     if (lane < 8) dd.mask[lane >> 2][lane & 3] = word;
@@ -159,33 +205,35 @@ struct Producer {
       dd.j0[0] = j0a;
       dd.j0[1] = j0b;
     }
-    __threadfence_block();
+    // __syncwarp orders the lanes' descriptor writes before lane 0's
+    // release-arrive on k_full; no further fence is needed
     __syncwarp();
     if (lane == 0) {
-      issued[stage] = t;
       uint8_t* kb = smem + C::kOffK + stage * C::kKVBytes;
-      uint8_t* vb = smem + C::kOffV + stage * C::kKVBytes;
       mbar_arrive_expect_tx(&k_full[stage], C::kKVBytes);
+      if (j0b == j0a + 64) {
 #pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
-        tma_load_2d(kb + h * C::kRegion, tmK, &k_full[stage], 64 * h, kv_row0 + j0a);
-        tma_load_2d(kb + h * C::kRegion + 8192, tmK, &k_full[stage], 64 * h, kv_row0 + j0b);
-      }
-      mbar_arrive_expect_tx(&v_full[stage], C::kKVBytes);
+        for (int h = 0; h < D / 64; ++h) tma_load_2d(kb + h * C::kRegion, tmK2, &k_full[stage], 64 * h, kv_row0 + j0a);
+      } else {
 #pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
-        tma_load_2d(vb + h * C::kRegion, tmV, &v_full[stage], 64 * h, kv_row0 + j0a);
-        tma_load_2d(vb + h * C::kRegion + 8192, tmV, &v_full[stage], 64 * h, kv_row0 + j0b);
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_2d(kb + h * C::kRegion, tmK, &k_full[stage], 64 * h, kv_row0 + j0a);
+          tma_load_2d(kb + h * C::kRegion + 8192, tmK, &k_full[stage], 64 * h, kv_row0 + j0b);
+        }
       }
     }
+    emit_v_lag();  // V of the previous tile
     ++t;
+    vj0[0] = j0a;
+    vj0[1] = j0b;
   }
 
-  // A gathered tile of the first cnt staged columns (1 <= cnt <= 128).
+  // A gathered tile of the first cnt staged columns (1 <= cnt <= 128); its K
+  // and V rows are copied together.
   __device__ void emit_gather(int cnt) {
     if (!ok) return;
     int stage;
-    if (!acquire(stage)) return;
+    if (!acquire_k(stage)) return;
     TileDesc& dd = desc[stage];
     int any_late = 0;
 #pragma unroll
@@ -207,12 +255,14 @@ struct Producer {
       dd.kind = KIND_GATHER;
       dd.flags = F_MASK | (any_late ? F_CAUSAL : 0);
     }
-    __threadfence_block();
     __syncwarp();
+    emit_v_lag();  // V of the previous tile
+    int vstage;
+    if (!acquire_v(t, vstage)) return;
     // cp.async gather of 128 K and V rows into the 128B-swizzled layout.
     constexpr int CH = D * 2 / 16;  // 16-byte chunks per row
     const uint32_t kb = smem_u32(smem + C::kOffK + stage * C::kKVBytes);
-    const uint32_t vb = smem_u32(smem + C::kOffV + stage * C::kKVBytes);
+    const uint32_t vb = smem_u32(smem + C::kOffV + vstage * C::kKVBytes);
 #pragma unroll 4
     for (int it = 0; it < 128 * CH / 32; ++it) {
       const int idx = it * 32 + lane;
@@ -224,7 +274,6 @@ struct Producer {
       cp_async16(vb + off, Vh + (size_t)j * D + q * 8);
     }
     cp_async_commit();
-    if (lane == 0) issued[stage] = t;
     // signal the previous gathered tile, keep this one in flight
     if (pending >= 0) {
       cp_async_wait<1>();
@@ -235,23 +284,23 @@ struct Producer {
         mbar_arrive(&v_full[pending]);
       }
     }
-    pending = stage;
+    pending = stage;  // K and V slots of a tile have the same index
     ++t;
+    ++tv;
   }
 
   __device__ void emit_end() {
+    emit_v_lag();
     flush_pending();
-    for (int e = 0; e < 2 && ok; ++e) {
-      int stage;
-      if (!acquire(stage)) return;
-      if (lane == 0) {
-        desc[stage].kind = KIND_END;
-        issued[stage] = -1;
-        mbar_arrive(&k_full[stage]);
-      }
-      __syncwarp();
-      ++t;
+    if (!ok) return;
+    int stage;
+    if (!acquire_k(stage)) return;
+    if (lane == 0) {
+      desc[stage].kind = KIND_END;
+      mbar_arrive(&k_full[stage]);
     }
+    __syncwarp();
+    ++t;  // the END tile has no V side: tv stays at the last real tile
   }
 
   // Appends a warp-wide batch of candidate columns to the staging list,
@@ -286,19 +335,20 @@ struct Producer {
   }
 
   // Waits (bounded, ignoring the abort flag) until every copy this producer
-  // started has landed, so that the CTA never exits with copies in flight.
+  // started has landed, so that the CTA never exits with copies in flight:
+  // the last kStages tiles of each ring (older ones were waited for when
+  // their slots were reused).  The slots carry no per-stage bookkeeping
+  // (an array indexed by stage would move the producer's state to local
+  // memory).
   __device__ void drain() {
     cp_async_wait<0>();
     __syncwarp();
     if (lane == 0) {
       int dummy = 0;
-      for (int s = 0; s < C::kStages; ++s) {
-        if (issued[s] >= 0) {
-          const uint32_t par = (issued[s] / C::kStages) & 1;
-          mbar_wait(&k_full[s], par, &dummy, st, 9);
-          mbar_wait(&v_full[s], par, &dummy, st, 9);
-        }
-      }
+      for (int u = max(0, t - C::kStages); u < t; ++u)
+        mbar_wait(&k_full[u % C::kStages], (u / C::kStages) & 1, &dummy, st, 9);
+      for (int u = max(0, tv - C::kStages); u < tv; ++u)
+        mbar_wait(&v_full[u % C::kStages], (u / C::kStages) & 1, &dummy, st, 9);
     }
     __syncwarp();
   }
@@ -354,6 +404,9 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi
       const int x0 = R + 64 * hh - j0 + 63 - 32 * wd;
       return __brev(wmap_window(W, x0 - 31)) & count_mask(cnt, wd);
     };
+    // The words of a group's later tiles are fetched four tiles at a time,
+    // one word per lane, and the next four are requested while the current
+    // ones are emitted, so that no tile waits for a bitmap load.
     for (int base = top; base >= 0 && P.ok; base -= 32) {
       const int gl = base - lane;
       int lo_l = 0, hi_l = -1;
@@ -373,16 +426,37 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi
       for (int k = 0; k < nbatch && P.ok; ++k) {
         const int lo_key = __shfl_sync(0xFFFFFFFFu, lo_l, k);
         const int hi_key = __shfl_sync(0xFFFFFFFFu, hi_l, k);
-        uint32_t word = 0xFFFFFFFFu;
+        uint32_t wf = 0xFFFFFFFFu;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const uint32_t v = __shfl_sync(0xFFFFFFFFu, w8[q], k);
-          if (lane == q) word = v;
+          if (lane == q) wf = v;
         }
-        for (int j0 = lo_key; j0 <= hi_key && P.ok; j0 += 128) {
+        const int ntile = (hi_key - lo_key) / 128 + 1;
+        // word (lane & 7) of tile 1 + 4c + (lane >> 3)
+        auto chunk_word = [&](int c) -> uint32_t {
+          const int tt = 1 + 4 * c + (lane >> 3);
+          if (tt >= ntile) return 0xFFFFFFFFu;
+          const int j0 = lo_key + 128 * tt;
+          return tile_word(j0, min(128, hi_key - j0 + 1), (lane >> 2) & 1, lane & 3);
+        };
+        uint32_t wcur = (ntile > 1) ? chunk_word(0) : 0xFFFFFFFFu;
+        uint32_t wnext = (ntile > 5) ? chunk_word(1) : 0xFFFFFFFFu;
+        {
+          const int cnt = min(128, hi_key - lo_key + 1);
+          P.emit_range(lo_key, lo_key + 64, wf, (lo_key + cnt - 1 > R) ? F_CAUSAL : 0);
+        }
+        for (int tt = 1; tt < ntile && P.ok; ++tt) {
+          const int slot = (tt - 1) & 3;
+          if (slot == 0 && tt > 1) {
+            wcur = wnext;
+            const int c = (tt - 1) >> 2;
+            wnext = (1 + 4 * (c + 1) < ntile) ? chunk_word(c + 1) : 0xFFFFFFFFu;
+          }
+          const uint32_t wv = __shfl_sync(0xFFFFFFFFu, wcur, slot * 8 + (lane & 7));
+          const int j0 = lo_key + 128 * tt;
           const int cnt = min(128, hi_key - j0 + 1);
-          if (j0 != lo_key && lane < 8) word = tile_word(j0, cnt, lane >> 2, lane & 3);
-          P.emit_range(j0, j0 + 64, word, (j0 + cnt - 1 > R) ? F_CAUSAL : 0);
+          P.emit_range(j0, j0 + 64, lane < 8 ? wv : 0xFFFFFFFFu, (j0 + cnt - 1 > R) ? F_CAUSAL : 0);
         }
       }
     }
@@ -486,7 +560,8 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi
 template <int D, int POL>
 __global__ void __launch_bounds__(320, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
+                const __grid_constant__ CUtensorMap tmV2, const AttnParams p) {
   using C = AttnCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
@@ -504,11 +579,12 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
   uint64_t* k_full = bars;
   uint64_t* v_full = bars + C::kStages;
-  uint64_t* kv_empty = bars + 2 * C::kStages;
-  uint64_t* s_full = bars + 3 * C::kStages;
+  uint64_t* k_empty = bars + 2 * C::kStages;  // S = Q K^T of the slot's tile is done
+  uint64_t* v_empty = bars + 3 * C::kStages;  // P V of the slot's tile is done
+  uint64_t* d_empty = bars + 4 * C::kStages;  // the softmax warps have read the descriptor
+  uint64_t* s_full = bars + 5 * C::kStages;
   uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* q_full = o_done + 2;
+  uint64_t* q_full = p_full + 2;
   uint64_t* mma_done = q_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -526,12 +602,13 @@ __global__ void __launch_bounds__(320, 1)
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
+      mbar_init(&d_empty[s], 256);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&s_full[w], 1);
-      mbar_init(&p_full[w], 128);
-      mbar_init(&o_done[w], 1);
+      mbar_init(&p_full[w], 256);
     }
     mbar_init(q_full, 1);
     mbar_init(mma_done, 1);
@@ -556,9 +633,13 @@ __global__ void __launch_bounds__(320, 1)
     P.sbits = smem + C::kOffSBits;
     P.k_full = k_full;
     P.v_full = v_full;
-    P.kv_empty = kv_empty;
+    P.k_empty = k_empty;
+    P.v_empty = v_empty;
+    P.d_empty = d_empty;
     P.tmK = &tmK;
     P.tmV = &tmV;
+    P.tmK2 = &tmK2;
+    P.tmV2 = &tmV2;
     P.kv_row0 = (b * p.Hkv + kvh) * p.N;
     P.Kh = p.K + (size_t)P.kv_row0 * D;
     P.Vh = p.V + (size_t)P.kv_row0 * D;
@@ -566,8 +647,9 @@ __global__ void __launch_bounds__(320, 1)
     P.N = p.N;
     P.lane = lane;
     P.t = 0;
+    P.tv = 0;
+    P.vj0[0] = P.vj0[1] = 0;
     P.pending = -1;
-    for (int s = 0; s < C::kStages; ++s) P.issued[s] = -1;
     P.abort = abort;
     P.st = p.status;
     P.ok = true;
@@ -575,6 +657,8 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      prefetch_tmap(&tmK2);
+      prefetch_tmap(&tmV2);
       mbar_arrive_expect_tx(q_full, C::kQBytes);
       const int qrow = (b * p.Hq + head) * p.N + R;
 #pragma unroll
@@ -599,21 +683,23 @@ __global__ void __launch_bounds__(320, 1)
     // --------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t qaddr = smem_u32(smem + C::kOffQ);
+      // O_0 += P[:, 0:64] V[0:64, :] and O_1 += P[:, 64:128] V[64:128, :];
+      // warpgroup w's bf16 P occupies TMEM columns 64w .. 64w+31 of the buffer
       auto issue_pv = [&](int tp) -> bool {
-        const int wp = tp & 1;
+        const int bp = tp & 1;
         const int sp = tp % C::kStages;
-        if (!mbar_wait(&p_full[wp], (tp >> 1) & 1, abort, p.status, 3)) return false;
+        if (!mbar_wait(&p_full[bp], (tp >> 1) & 1, abort, p.status, 3)) return false;
         if (!mbar_wait(&v_full[sp], (tp / C::kStages) & 1, abort, p.status, 4)) return false;
         tc_fence_after();
         const uint32_t vaddr = smem_u32(smem + C::kOffV + sp * C::kKVBytes);
-        const uint32_t d_tmem = tmem + (wp ? C::kColO1 : C::kColO0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, C::kRegion, 1024);
-          umma_ts(d_tmem, tmem + wp * 128 + kk * 8, bd, C::kIdescPV, (tp >= 2 || kk > 0) ? 1u : 0u);
+          const uint32_t d_tmem = tmem + (kk < 4 ? C::kColO0 : C::kColO1);
+          const uint32_t a_tmem = tmem + bp * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+          umma_ts(d_tmem, a_tmem, bd, C::kIdescPV, (tp > 0 || (kk & 3) > 0) ? 1u : 0u);
         }
-        umma_commit(&o_done[wp]);
-        umma_commit(&kv_empty[sp]);
+        umma_commit(&v_empty[sp]);
         return true;
       };
       bool ok = mbar_wait(q_full, 0, abort, p.status, 2);
@@ -625,7 +711,7 @@ __global__ void __launch_bounds__(320, 1)
         // Q and K were written by TMA or by cp.async plus the producer's proxy
         // fence; the barrier alone orders them before the MMA (no tcgen05
         // fence here: it would stall the issue of every tile).
-        const int w = t & 1;
+        const int w = t & 1;  // S buffer
         const uint32_t kaddr = smem_u32(smem + C::kOffK + st * C::kKVBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -635,6 +721,7 @@ __global__ void __launch_bounds__(320, 1)
           umma_ss(tmem + w * 128, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[w]);
+        umma_commit(&k_empty[st]);
         if (pend >= 0 && !issue_pv(pend)) { ok = false; pend = -1; break; }
         pend = t;
         ++t;
@@ -647,7 +734,7 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------- softmax
-    const int wg = warp >> 2;
+    const int wg = warp >> 2;  // column half of every tile
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const int i = R + r;
@@ -657,79 +744,82 @@ __global__ void __launch_bounds__(320, 1)
     float m_run = -INFINITY, l_run = 0.f;
     int n = 0;
     unsigned nnz = 0;
-    for (int t = wg;; t += 2) {
+    for (int t = 0;; ++t) {
       const int st = t % C::kStages;
       if (!warp_wait(&k_full[st], (t / C::kStages) & 1, abort, p.status, 10)) break;
       const TileDesc& dd = desc[st];
       const int kind = dd.kind;
       if (kind == KIND_END) break;
-      if (!warp_wait(&s_full[wg], n & 1, abort, p.status, 11)) break;
+      if (!warp_wait(&s_full[t & 1], (t >> 1) & 1, abort, p.status, 11)) break;
       tc_fence_after();
       const int flags = dd.flags;
-      // Membership words of this warp's 64-row half, one per 32-column chunk.
-      // All rows of a warp lie in one half, so the chunk tests are warp-uniform:
-      // full chunks need no masking, empty chunks are not exponentiated.
-      uint32_t mw[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+      const uint32_t scol = srow + (t & 1) * 128 + wg * 64;
+      // Membership words of this warp's 64-row half for the warpgroup's two
+      // 32-column chunks.  All rows of a warp lie in one half, so the chunk
+      // tests are warp-uniform: full chunks need no masking, empty chunks are
+      // not exponentiated.
+      uint32_t mw[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
       if (flags & F_MASK) {
-        const uint4 m4 = *reinterpret_cast<const uint4*>(&dd.mask[half][0]);
-        mw[0] = m4.x; mw[1] = m4.y; mw[2] = m4.z; mw[3] = m4.w;
+        const uint2 m2 = *reinterpret_cast<const uint2*>(&dd.mask[half][2 * wg]);
+        mw[0] = m2.x;
+        mw[1] = m2.y;
       }
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4)
-        tmem_ld32(srow + wg * 128 + c4 * 32, sr[c4]);
+      uint32_t sr[2][32];
+      tmem_ld32(scol, sr[0]);
+      tmem_ld32(scol + 32, sr[1]);
       tmem_wait_ld();
+      reg_fence(sr[0]);
+      reg_fence(sr[1]);
+      float s[64];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) reg_fence(sr[c4]);
-      float s[128];
+      for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
 #pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        if (mw[c4] != 0xFFFFFFFFu && mw[c4] != 0u) {
+      for (int c2 = 0; c2 < 2; ++c2) {
+        if (mw[c2] != 0xFFFFFFFFu && mw[c2] != 0u) {
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            if (!((mw[c4] >> e) & 1u)) s[c4 * 32 + e] = -INFINITY;
+            if (!((mw[c2] >> e) & 1u)) s[c2 * 32 + e] = -INFINITY;
         }
       }
       if (flags & (F_CAUSAL | F_ASHAPE)) {
         const bool causal = flags & F_CAUSAL;
         const bool ash = flags & F_ASHAPE;
         if (kind == KIND_RANGE) {
-          const int ja = dd.j0[0], jb = dd.j0[1];
+          const int jw = dd.j0[wg];
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const int j = ((c < 64) ? ja : jb) + (c & 63);
+          for (int c = 0; c < 64; ++c) {
+            const int j = jw + c;
             bool drop = causal && (j > i);
             drop |= ash && (j >= p.n_sink) && (i - j >= p.n_local);
             if (drop) s[c] = -INFINITY;
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const int j = dd.cols[c];
+          for (int c = 0; c < 64; ++c) {
+            const int j = dd.cols[wg * 64 + c];
             if (causal && j > i) s[c] = -INFINITY;
           }
         }
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          if (mw[c4] != 0u) {
+        for (int c2 = 0; c2 < 2; ++c2) {
+          if (mw[c2] != 0u) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) nnz += (s[c4 * 32 + e] != -INFINITY);
+            for (int e = 0; e < 32; ++e) nnz += (s[c2 * 32 + e] != -INFINITY);
           }
         }
       } else {
-        nnz += __popc(mw[0]) + __popc(mw[1]) + __popc(mw[2]) + __popc(mw[3]);
+        nnz += __popc(mw[0]) + __popc(mw[1]);
       }
+      mbar_arrive(&d_empty[st]);  // descriptor no longer read
       // row max: eight independent chains over the non-empty chunks
       float mx8[8];
 #pragma unroll
       for (int k8 = 0; k8 < 8; ++k8) mx8[k8] = -INFINITY;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        if (mw[c4] != 0u) {
+      for (int c2 = 0; c2 < 2; ++c2) {
+        if (mw[c2] != 0u) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[c4 * 32 + e]);
+          for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[c2 * 32 + e]);
         }
       }
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
@@ -742,18 +832,18 @@ __global__ void __launch_bounds__(320, 1)
         m_run = m_new;
       }
       const float msub = (m_run == -INFINITY) ? 0.f : m_run;
-      // P = 2^(s * scale * log2 e - m) as bf16 pairs over S's columns; the
-      // argument and the row sum use packed two-lane fp32 instructions.
+      // P = 2^(s * scale * log2 e - m) as bf16 pairs; the argument and the
+      // row sum use packed two-lane fp32 instructions.
       const uint64_t sl2x2 = f32x2_pack(sl2, sl2), nm2 = f32x2_pack(-msub, -msub);
       uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c2 = 0; c2 < 2; ++c2) {
         uint32_t pk[16];
-        if (mw[c4] != 0u) {
+        if (mw[c2] != 0u) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             float x0, x1;
-            f32x2_unpack(f32x2_fma(f32x2_pack(s[c4 * 32 + e], s[c4 * 32 + e + 1]), sl2x2, nm2), x0, x1);
+            f32x2_unpack(f32x2_fma(f32x2_pack(s[c2 * 32 + e], s[c2 * 32 + e + 1]), sl2x2, nm2), x0, x1);
             const float p0 = fast_exp2(x0);
             const float p1 = fast_exp2(x1);
             acc2[(e >> 1) & 1] = f32x2_add(acc2[(e >> 1) & 1], f32x2_pack(p0, p1));
@@ -763,7 +853,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = 0u;
         }
-        tmem_st16(srow + wg * 128 + c4 * 16, pk);
+        tmem_st16(scol + c2 * 16, pk);
       }
       float a0, a1, b0, b1;
       f32x2_unpack(acc2[0], a0, a1);
@@ -772,7 +862,8 @@ __global__ void __launch_bounds__(320, 1)
       // lazy correction of the running output (rare after the first tiles),
       // done after the P stores so that the scores are no longer live
       if (__any_sync(0xFFFFFFFFu, resc && n > 0)) {
-        if (!warp_wait(&o_done[wg], (n - 1) & 1, abort, p.status, 12)) break;
+        // P V of the previous tile must be complete before O is rescaled
+        if (!warp_wait(&v_empty[(n - 1) % C::kStages], ((n - 1) / C::kStages) & 1, abort, p.status, 12)) break;
         tc_fence_after();
         const uint32_t orow = srow + (wg ? C::kColO1 : C::kColO0);
 #pragma unroll 1
@@ -788,7 +879,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[wg]);
+      mbar_arrive(&p_full[t & 1]);
       ++n;
     }
     // ----------------------------------------------------------- epilogue
@@ -799,7 +890,7 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) atomicAdd(&p.status->nnz, c);
     }
     bool ok = !*abort;
-    if (ok && n > 0) ok = warp_wait(&o_done[wg], (n - 1) & 1, abort, p.status, 13);
+    if (ok && n > 0) ok = warp_wait(&v_empty[(n - 1) % C::kStages], ((n - 1) / C::kStages) & 1, abort, p.status, 13);
     named_bar_sync(1, 256);
     float* xch = reinterpret_cast<float*>(smem + C::kOffK);  // all S MMAs are done: K stage 0 is free
     xch[(wg * 128 + r) * 4 + 0] = m_run;
@@ -859,20 +950,21 @@ __global__ void __launch_bounds__(320, 1)
 // ------------------------------------------------------------------ launch
 template <int D, int POL>
 static cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                               const AttnParams& p, cudaStream_t stream) {
+                               const CUtensorMap& tk2, const CUtensorMap& tv2, const AttnParams& p,
+                               cudaStream_t stream) {
   using C = AttnCfg<D>;
   auto kfn = attn_kernel<D, POL>;
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.N / 128, p.nh, p.B);
-  kfn<<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+  kfn<<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, tk2, tv2, p);
   return cudaGetLastError();
 }
 
 cudaError_t attn_dispatch(int d, int pol, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const AttnParams& p, cudaStream_t stream) {
+                          const CUtensorMap& tk2, const CUtensorMap& tv2, const AttnParams& p, cudaStream_t stream) {
 #define MINF_CASE(DD, PP) \
-  if (d == DD && pol == PP) return launch_attn<DD, PP>(tq, tk, tv, p, stream);
+  if (d == DD && pol == PP) return launch_attn<DD, PP>(tq, tk, tv, tk2, tv2, p, stream);
   MINF_CASE(64, POL_DENSE)
   MINF_CASE(64, POL_ASHAPE)
   MINF_CASE(64, POL_VS)

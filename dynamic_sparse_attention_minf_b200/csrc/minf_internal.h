@@ -42,8 +42,10 @@ struct AttnParams {
   DevStatus* status;
 };
 
+// tq: Q with 128-row boxes; tk/tv: K and V with 64-row boxes; tk2/tv2: K and V
+// with 128-row boxes (all 128-byte swizzled, 64 columns wide)
 cudaError_t attn_dispatch(int d, int pol, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const AttnParams& p, cudaStream_t stream);
+                          const CUtensorMap& tk2, const CUtensorMap& tv2, const AttnParams& p, cudaStream_t stream);
 
 // ---- estimation / index kernels (estimate.cu, index.cu)
 struct VsEstParams {

@@ -71,7 +71,8 @@ LAUNCHES_PER_STEP = 6 + 3 + 1 + 3 + 1 + 1
 def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None, marks=None):
     """Estimation, index build and sparse attention for every head of the
     layer, in stream order; O (and LSE) are filled head by head.  ``marks``
-    (optional) gets ``mark(name)`` calls around the attention launches."""
+    (optional) gets ``mark(name)`` calls, ``<phase>:pre`` and ``<phase>:post``,
+    around every call of the layer."""
     mark = marks.mark if marks is not None else (lambda name: None)
     w, b = plan.w, plan.bufs
     shp = plan.shape
@@ -80,13 +81,17 @@ def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None, marks=None):
     P = minf._p
     if plan.vs_heads is not None:
         nv = plan.vs_heads.numel()
+        mark("vs_est:pre")
         minf._check("minf_estimate_vs", L.minf_estimate_vs(
             minf.ctypes.byref(shp), P(q), P(k), P(plan.vs_heads), nv, w.last_q, w.k_v, w.k_s,
             P(b["v_idx"]), P(b["s_idx"]), None, None, P(b["ws_vs_est"]), b["ws_vs_est"].numel(), st))
+        mark("vs_est:post")
         ic = b["vs_index"].c()
+        mark("vs_index:pre")
         minf._check("minf_build_index", L.minf_build_index(
             minf.ctypes.byref(shp), nv, P(b["v_idx"]), w.k_v, P(b["s_idx"]), w.k_s, minf.ctypes.byref(ic),
             P(b["ws_vs_idx"]), b["ws_vs_idx"].numel(), st))
+        mark("vs_index:post")
         mark("vs_attn:pre")
         minf._check("minf_sparse_attn_vs", L.minf_sparse_attn_vs(
             minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.vs_heads), nv, minf.ctypes.byref(ic),
@@ -94,17 +99,23 @@ def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None, marks=None):
         mark("vs_attn:post")
     if plan.bs_heads is not None:
         nbh = plan.bs_heads.numel()
+        mark("bs_est:pre")
         minf._check("minf_estimate_bs", L.minf_estimate_bs(
             minf.ctypes.byref(shp), P(q), P(k), P(plan.bs_heads), nbh, w.block, w.k_b,
             P(b["blk_idx"]), P(b["blk_cnt"]), None, P(b["ws_bs_est"]), b["ws_bs_est"].numel(), st))
+        mark("bs_est:post")
+        mark("bs_attn:pre")
         minf._check("minf_sparse_attn_bs", L.minf_sparse_attn_bs(
             minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.bs_heads), nbh, P(b["blk_idx"]),
             P(b["blk_cnt"]), w.k_b, P(o), P(lse), P(b["ws_bs_attn"]), b["ws_bs_attn"].numel(), st))
+        mark("bs_attn:post")
     if plan.a_heads is not None:
         na = plan.a_heads.numel()
+        mark("a_attn:pre")
         minf._check("minf_attn_ashape", L.minf_attn_ashape(
             minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.a_heads), na, w.n_sink, w.n_local,
             P(o), P(lse), P(b["ws_a"]), b["ws_a"].numel(), st))
+        mark("a_attn:post")
     return o, lse
 
 
