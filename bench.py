@@ -95,6 +95,30 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(lines)}
 
 
+_KERNEL_SOURCES = ("csrc/attn.cu", "csrc/minf_device.cuh", "csrc/minf_internal.h")
+_TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "attn_vs_llama3_8b_layer_n1m_dram.md")
+
+
+def _recorded_traffic():
+    """DRAM bytes (read + write) of one Vertical-Slash attention launch of the
+    1M layer, from the committed ncu summary, or None when the attention
+    sources no longer hash to the ones that summary was captured from."""
+    import hashlib
+    try:
+        text = open(_TRAFFIC_PROFILE).read()
+        h = hashlib.sha256()
+        for f in _KERNEL_SOURCES:
+            with open(os.path.join(ROOT, "dynamic_sparse_attention_minf_b200", f), "rb") as fh:
+                h.update(fh.read())
+        vals = dict(line.split(": ", 1) for line in text.splitlines()
+                    if line.startswith(("traffic_bytes_per_launch: ", "kernel_sources_sha256: ")))
+        if vals.get("kernel_sources_sha256", "").strip() != h.hexdigest():
+            return None
+        return float(vals["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws > 1:
@@ -368,7 +392,9 @@ def run_ours(args, dist, rank, world, local):
         "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None,
         "roofline": {"kernel": "attn_kernel<128, vertical_slash>", "bound": "tensor",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "frac": (achieved / peak) if achieved else None,
+                     "traffic": (_recorded_traffic() if w.N == 1 << 20 else None),
+                     "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                      "peak_source": f"{src} bf16_tflops_sustained", "ms_per_launch": vs_ms,
                      "executed_tflop_per_launch": vs_exec / 1e12},
         "e2e": {"value": _throughput(world, useful, e2e_ms), "unit": "TFLOP/s",

@@ -196,3 +196,31 @@ def test_bs_all_blocks_equals_dense():
     od, ld = minf.minf_dense_attn(q, k, v)
     assert (o.float() - od.float()).abs().max().item() <= 1e-2
     assert (lse - ld).abs().max().item() <= 1e-3
+
+
+# -------------------------------------------------------------- edge cases
+def test_vs_offset_zero_and_one_vertical():
+    """k_s = 1 keeps only the forced offset 0 (block-diagonal bands) and k_v = 1 one column."""
+    w = wl.small(Hq=2, Hkv=1, N=1024, d=64, seed=31, k_v=1, k_s=1)
+    gv, gs = _vs_pipeline(w, [0, 1])
+    assert (gs == 0).all()
+
+
+def test_bs_diagonal_block_only():
+    """k_b = 1: every query block attends to its own (forced) diagonal block only."""
+    w = wl.small(Hq=2, Hkv=1, N=1024, d=128, seed=32, bias="block", patterns=[wl.PAT_BS] * 2, k_b=1)
+    _bs_pipeline(w, [0, 1])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_minimum_size_one_tile(d):
+    """N = 128: one query tile, one key tile, for every pattern."""
+    w = wl.small(Hq=2, Hkv=1, N=128, d=d, seed=33, k_v=16, k_s=8)
+    _vs_pipeline(w, [0, 1])
+    wb = wl.small(Hq=2, Hkv=1, N=128, d=d, seed=34, bias="block", patterns=[wl.PAT_BS] * 2, k_b=2)
+    _bs_pipeline(wb, [0, 1])
+    q, k, v, qn, kn, vn = _inputs(w)
+    o, lse = minf.minf_attn_ashape(q, k, v, [0, 1], 16, 32)
+    _check_attn(o, lse, qn, kn, vn, [0, 1], w, lambda hi, h: (lambda r: orc.mask_ashape(r, w.N, 16, 32)))
+    o, lse = minf.minf_dense_attn(q, k, v)
+    _check_attn(o, lse, qn, kn, vn, [0, 1], w, lambda hi, h: (lambda r: orc.mask_dense(r, w.N)))
