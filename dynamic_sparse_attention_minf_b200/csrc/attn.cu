@@ -844,8 +844,14 @@ __global__ void __launch_bounds__(320, 1)
           for (int e = 0; e < 32; e += 2) {
             float x0, x1;
             f32x2_unpack(f32x2_fma(f32x2_pack(s[c2 * 32 + e], s[c2 * 32 + e + 1]), sl2x2, nm2), x0, x1);
-            const float p0 = fast_exp2(x0);
-            const float p1 = fast_exp2(x1);
+            // one pair in four on the FMA pipe, the rest on the MUFU
+            float p0, p1;
+            if ((e & 6) == 6) {
+              exp2_poly_x2(x0, x1, p0, p1);
+            } else {
+              p0 = fast_exp2(x0);
+              p1 = fast_exp2(x1);
+            }
             acc2[(e >> 1) & 1] = f32x2_add(acc2[(e >> 1) & 1], f32x2_pack(p0, p1));
             pk[e >> 1] = pack_bf16x2(p0, p1);
           }
