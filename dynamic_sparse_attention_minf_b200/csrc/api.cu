@@ -212,7 +212,7 @@ minf_status minf_estimate_vs(const minf_shape* s, const minf_bf16* Q, const minf
   cudaStream_t cs = (cudaStream_t)stream;
   CUtensorMap tq, tk;
   if (((uintptr_t)Q | (uintptr_t)K) & 15) return MINF_ERR_INVALID_ARG;
-  if (!make_map(&tq, Q, (long long)s->B * s->Hq * s->N, s->d, 128) ||
+  if (!make_map(&tq, Q, (long long)s->B * s->Hq * s->N, s->d, 64) ||
       !make_map(&tk, K, (long long)s->B * s->Hkv * s->N, s->d, 64))
     return MINF_ERR_CUDA;
   cudaError_t e = vs_estimate_tc_launch(tq, tk, p, cs);

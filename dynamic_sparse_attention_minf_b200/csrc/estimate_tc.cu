@@ -3,20 +3,22 @@
 //
 // One CTA takes one head and a run of 128-key tiles.  The scores of the last
 // query rows against a key tile, S = Q_last K^T, are one tcgen05 GEMM (bf16
-// inputs, exact products, fp32 accumulation in TMEM).  Q's last 128 rows are
-// the A operand; the real rows are the last `last_q` <= 64 of them, in TMEM
-// lanes 64..127, read by warps 2, 3, 6, 7 (two threads per row, 64 columns
-// each).  K tiles stream through a 3-stage TMA ring.
+// inputs, exact products, fp32 accumulation in TMEM).  The A operand holds
+// Q's last 64 rows twice (rows 0-63 and 64-127), so that every TMEM lane
+// quarter holds real scores: lanes 0-63 serve key columns 0-63 and lanes
+// 64-127 key columns 64-127, and all eight score warps (two per SM
+// sub-partition) work on each tile, 32 rows x 32 columns each.  The real rows
+// are the last `last_q` <= 64.  K tiles stream through a 3-stage TMA ring.
 //
 //  pass 1: each thread keeps an online (max, sum) of 2^(s * scale * log2 e)
-//          over its columns of the CTA's tiles; the two halves of a row are
-//          merged and written as the CTA's partial of that row.
+//          over its columns of the CTA's tiles; the four column groups of a
+//          row are merged and written as the CTA's partial of that row.
 //  pass 2: p = 2^(x - m) / l with the combined row statistics is written to
-//          shared memory, and 128 threads form, in a fixed order, the column
+//          shared memory, and the CTA forms, in a fixed order, the column
 //          sums (vertical scores) and the tile's 191 diagonal partials.
 //
-// warp 0 lane 0: TMA producer; warp 1: TMEM owner and MMA issuer;
-// warps 2, 3, 6, 7: score warps; warps 4, 5 idle.
+// warps 0-7: score warps; warp 8 lane 0: TMA producer; warp 9: TMEM owner and
+// MMA issuer.
 #include <algorithm>
 
 #include "minf_device.cuh"
@@ -26,9 +28,10 @@ namespace minf {
 
 template <int D>
 struct EstCfg {
-  static constexpr int kThreads = 256;
+  static constexpr int kThreads = 320;
+  static constexpr int kScoreThreads = 256;
   static constexpr int kRegion = 128 * 128;
-  static constexpr int kTileBytes = 128 * D * 2;  // 128 rows (Q) or 128 keys (K)
+  static constexpr int kTileBytes = 128 * D * 2;  // 128 rows (Q twice) or 128 keys (K)
   static constexpr int kStages = 3;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTileBytes;
@@ -39,14 +42,14 @@ struct EstCfg {
   // barriers: q_full, k_full[3], k_empty[3], s_full[2], s_free[2], mma_done
   static constexpr int kNumBars = 1 + 2 * kStages + 4 + 1;
   static constexpr int kOffMisc = kOffBars + kNumBars * 8;
-  static constexpr int kOffXch = kOffMisc + 16;             // pass 1: [2][64][2] fp32
-  static constexpr int kSmem = kOffXch + 2 * 64 * 2 * 4;
+  static constexpr int kOffXch = kOffMisc + 16;             // pass 1: [4][64][2] fp32
+  static constexpr int kSmem = kOffXch + 4 * 64 * 2 * 4;
   static_assert(kSmem <= 232448, "shared memory budget");
   static constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);
 };
 
 template <int D, int PASS>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(320, 1)
     vs_est_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const VsEstParams p, int tiles_per_cta, int nchunks) {
   using C = EstCfg<D>;
@@ -82,13 +85,13 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&s_full[w], 1);
-      mbar_init(&s_free[w], 128);
+      mbar_init(&s_free[w], C::kScoreThreads);
     }
     mbar_init(mma_done, 1);
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
@@ -97,13 +100,17 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // Q's last 64 rows into rows 0-63 and again into rows 64-127
       mbar_arrive_expect_tx(q_full, C::kTileBytes);
-      const int qrow0 = (b * p.Hq + head) * p.N + p.N - 128;
+      const int qrow0 = (b * p.Hq + head) * p.N + p.N - 64;
 #pragma unroll
-      for (int h = 0; h < D / 64; ++h) tma_load_2d(smem + C::kOffQ + h * C::kRegion, &tmQ, q_full, 64 * h, qrow0);
+      for (int h = 0; h < D / 64; ++h) {
+        tma_load_2d(smem + C::kOffQ + h * C::kRegion, &tmQ, q_full, 64 * h, qrow0);
+        tma_load_2d(smem + C::kOffQ + h * C::kRegion + 8192, &tmQ, q_full, 64 * h, qrow0);
+      }
       const int kv_row0 = (b * p.Hkv + kvh) * p.N;
       int issued = 0;
       for (int k = 0; k < nt; ++k) {
@@ -124,7 +131,7 @@ __global__ void __launch_bounds__(256, 1)
         mbar_wait(&k_full[k % C::kStages], (k / C::kStages) & 1, &dummy, p.status, 62);
       mbar_wait(q_full, 0, &dummy, p.status, 63);
     }
-  } else if (warp == 1) {
+  } else if (warp == 9) {
     // --------------------------------------------------------- MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(q_full, 0, abort, p.status, 64);
@@ -150,16 +157,14 @@ __global__ void __launch_bounds__(256, 1)
       mbar_wait(mma_done, 0, &dummy, p.status, 67);
     }
     __syncwarp();
-  } else if ((warp & 3) >= 2) {
+  } else {
     // ------------------------------------------------------- score warps
-    const int qq = warp & 3;          // TMEM lane quarter 2 or 3: rows 64..127 of the Q tile
-    const int hc = warp >> 2;         // key columns 64 hc .. 64 hc + 63 of every tile
-    const int r = qq * 32 + lane;
-    const int qrow = r - 64;          // query row N - 64 + qrow
-    const int i = p.N - 128 + r;
-    const bool real = r >= 128 - p.last_q;
-    const int ctid = (hc * 2 + (qq - 2)) * 32 + lane;
-    const uint32_t taddr = tmem + ((uint32_t)(qq * 32) << 16) + hc * 64;
+    const int qq = warp & 3;                      // TMEM lane quarter
+    const int grp = (qq >> 1) * 2 + (warp >> 2);  // column group: key columns 32 grp .. 32 grp + 31
+    const int qrow = (qq & 1) * 32 + lane;        // query row N - 64 + qrow
+    const int i = p.N - 64 + qrow;
+    const bool real = qrow >= 64 - p.last_q;
+    const uint32_t taddr = tmem + ((uint32_t)(qq * 32) << 16) + grp * 32;
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     float mr = 0.f, il = 0.f;
@@ -169,74 +174,94 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int k = 0; k < nt; ++k) {
       const int buf = k & 1;
-      // all four score warps agree before going on (pass 2 meets at a
-      // barrier below, which a warp that gave up would never reach)
+      // all score warps agree before going on (pass 2 meets at a barrier
+      // below, which a warp that gave up would never reach)
       const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (k >> 1) & 1, abort, p.status, 68));
-      if (!bar_and(2, 128, got)) break;
+      if (!bar_and(2, C::kScoreThreads, got)) break;
       tc_fence_after();
-      uint32_t v0[32], v1[32];
+      uint32_t v0[32];
       tmem_ld32(taddr + buf * 128, v0);
-      tmem_ld32(taddr + buf * 128 + 32, v1);
       tmem_wait_ld();
       reg_fence(v0);
-      reg_fence(v1);
       tc_fence_before();
       mbar_arrive(&s_free[buf]);
-      const int j0 = (t0 + k) * 128 + hc * 64;
-      float x[64];
+      const int j0 = (t0 + k) * 128 + grp * 32;
+      float x[32];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float sv = __uint_as_float(c < 32 ? v0[c] : v1[c - 32]);
-        x[c] = (real && j0 + c <= i) ? sv * sl2 : -INFINITY;
-      }
+      for (int c = 0; c < 32; ++c) x[c] = (real && j0 + c <= i) ? __uint_as_float(v0[c]) * sl2 : -INFINITY;
       if (PASS == 1) {
-        float m8[8];
+        float m4[4];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+        for (int q = 0; q < 4; ++q) m4[q] = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], x[c]);
-        const float tm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int c = 0; c < 32; ++c) m4[c & 3] = fmaxf(m4[c & 3], x[c]);
+        const float tm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         if (tm > m) {
-          if (m != -INFINITY) l *= exp2f(m - tm);
+          if (m != -INFINITY) l *= fast_exp2(m - tm);
           m = tm;
         }
         if (m != -INFINITY) {
           float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < 64; ++c) a4[c & 3] += exp2f(x[c] - m);
+          for (int c = 0; c < 32; ++c) a4[c & 3] += fast_exp2(x[c] - m);
           l += (a4[0] + a4[1]) + (a4[2] + a4[3]);
         }
       } else {
         float* P = reinterpret_cast<float*>(smem + C::kOffP + buf * C::kPBytes);
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          P[qrow * C::kPStride + hc * 64 + c] = (x[c] == -INFINITY) ? 0.f : exp2f(x[c] - mr) * il;
-        named_bar_sync(1, 128);
-        const int jj = (t0 + k) * 128 + ctid;
-        float cs = 0.f;
-        for (int q = 0; q < 64; ++q) cs += P[q * C::kPStride + ctid];
-        if (jj < p.N) p.v_score[bh * p.N + jj] = cs;
-        for (int kd = ctid; kd < 191; kd += 128) {
-          float dsum = 0.f;
-          const int qlo = max(0, kd - 127), qhi = min(63, kd);
-          for (int q = qlo; q <= qhi; ++q) dsum += P[q * C::kPStride + (q - kd + 127)];
-          p.dpart[(bh * ntiles + t0 + k) * 192 + kd] = dsum;
+        for (int c = 0; c < 32; ++c)
+          P[qrow * C::kPStride + grp * 32 + c] = (x[c] == -INFINITY) ? 0.f : fast_exp2(x[c] - mr) * il;
+        named_bar_sync(1, C::kScoreThreads);
+        const int tid = threadIdx.x;  // 0 .. 255
+        // Fixed-order sums over the tile's 64 rows, each as four interleaved
+        // partial sums (rows q = 0, 1, 2, 3 mod 4) added in a fixed order.
+        // Threads 0-127: vertical score of key column tid, then (0-62) the
+        // diagonal 128 + tid; threads 128-255: the diagonal tid - 128.
+        // Diagonal kd holds the entries (q, q - kd + 127).
+        auto diag = [&](int kd) {
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          const int qhi = min(63, kd);
+          // entry (q, q - kd + 127) sits at q * (stride + 1) + 127 - kd
+          constexpr int kStep = C::kPStride + 1;
+          int q = max(0, kd - 127);
+          int x = q * kStep + 127 - kd;
+          for (; q + 3 <= qhi; q += 4, x += 4 * kStep) {
+            a0 += P[x];
+            a1 += P[x + kStep];
+            a2 += P[x + 2 * kStep];
+            a3 += P[x + 3 * kStep];
+          }
+          for (; q <= qhi; ++q, x += kStep) a0 += P[x];
+          p.dpart[(bh * ntiles + t0 + k) * 192 + kd] = (a0 + a1) + (a2 + a3);
+        };
+        if (tid < 128) {
+          float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 16
+          for (int q = 0; q < 64; ++q) a4[q & 3] += P[q * C::kPStride + tid];
+          const int jj = (t0 + k) * 128 + tid;
+          if (jj < p.N) p.v_score[bh * p.N + jj] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+          if (tid < 63) diag(128 + tid);
+        } else {
+          diag(tid - 128);
         }
       }
     }
     if (PASS == 1) {
       float* xch = reinterpret_cast<float*>(smem + C::kOffXch);
-      xch[(hc * 64 + qrow) * 2] = m;
-      xch[(hc * 64 + qrow) * 2 + 1] = l;
-      named_bar_sync(1, 128);
-      if (hc == 0) {
-        const float m1 = xch[(64 + qrow) * 2], l1 = xch[(64 + qrow) * 2 + 1];
-        const float M = fmaxf(m, m1);
+      xch[(grp * 64 + qrow) * 2] = m;
+      xch[(grp * 64 + qrow) * 2 + 1] = l;
+      named_bar_sync(1, C::kScoreThreads);
+      if (grp == 0) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) M = fmaxf(M, xch[(g * 64 + qrow) * 2]);
         float L = 0.f;
         if (M != -INFINITY) {
-          if (m != -INFINITY) L += l * exp2f(m - M);
-          if (m1 != -INFINITY) L += l1 * exp2f(m1 - M);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const float mg = xch[(g * 64 + qrow) * 2], lg = xch[(g * 64 + qrow) * 2 + 1];
+            if (mg != -INFINITY) L += lg * fast_exp2(mg - M);
+          }
         }
         float* out = p.part_ml + ((bh * nchunks + chunk) * 64 + qrow) * 2;
         out[0] = M;
@@ -246,7 +271,7 @@ __global__ void __launch_bounds__(256, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }

@@ -64,8 +64,8 @@ struct VsEstParams {
 cudaError_t vs_estimate_launch(const VsEstParams& p, cudaStream_t stream);
 cudaError_t vs_combine_launch(const VsEstParams& p, int nparts, cudaStream_t stream);
 cudaError_t vs_slash_launch(const VsEstParams& p, cudaStream_t stream);
-// tensor-core estimation: tq views Q as [rows, d] with 128-row boxes, tk views
-// K with 64-row boxes (both 128-byte swizzled)
+// tensor-core estimation: tq and tk view Q and K as [rows, d] with 64-row
+// boxes (128-byte swizzled)
 cudaError_t vs_estimate_tc_launch(const CUtensorMap& tq, const CUtensorMap& tk, const VsEstParams& p,
                                   cudaStream_t stream);
 
