@@ -399,7 +399,7 @@ def run_ours(args, dist, rank, world, local):
                      "executed_tflop_per_launch": vs_exec / 1e12},
         "e2e": {"value": _throughput(world, useful, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": layer.LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": layer.launches_per_step(plan) * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

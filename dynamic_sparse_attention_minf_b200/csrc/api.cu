@@ -83,6 +83,7 @@ minf_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MINF_OK : MIN
 struct VsEstWs {
   DevStatus* status;
   float *part_ml, *row_ml, *v_score, *s_score, *dpart;
+  uint32_t* topk;
 };
 size_t plan_vs_est(const minf_shape* s, int nh, char* ws, VsEstWs* out) {
   Carver c{ws, 0};
@@ -95,6 +96,7 @@ size_t plan_vs_est(const minf_shape* s, int nh, char* ws, VsEstWs* out) {
   w.v_score = c.take<float>(bh * s->N);
   w.s_score = c.take<float>(bh * s->N);
   w.dpart = c.take<float>(bh * ntiles * 192);
+  w.topk = c.take<uint32_t>(topk_scratch_words((int)bh));
   if (out) *out = w;
   return c.off;
 }
@@ -229,6 +231,7 @@ minf_status minf_estimate_vs(const minf_shape* s, const minf_bf16* Q, const minf
   t.out_idx = v_idx;
   t.out_cnt = nullptr;
   t.status = w.status;
+  t.scratch = w.topk;
   e = topk_rows_launch(t, cs);
   if (e != cudaSuccess) return MINF_ERR_CUDA;
   t.scores = p.s_score;
@@ -281,6 +284,7 @@ minf_status minf_estimate_bs(const minf_shape* s, const minf_bf16* Q, const minf
   t.out_idx = blk_idx;
   t.out_cnt = blk_cnt;
   t.status = w.status;
+  t.scratch = nullptr;
   return cuda_status(topk_rows_launch(t, cs));
 }
 

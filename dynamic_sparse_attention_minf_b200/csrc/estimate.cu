@@ -256,7 +256,8 @@ cudaError_t vs_estimate_launch(const VsEstParams& p, cudaStream_t stream) {
 
 // ================================================================ top-k rows
 constexpr int kTopkThreads = 1024;
-constexpr int kTopkItems = 4;
+constexpr int kTopkItems = 16;
+constexpr int kTopkLoads = 16;
 
 __device__ __forceinline__ uint32_t order_key(float x) {
   const uint32_t u = __float_as_uint(x);
@@ -291,13 +292,13 @@ __device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long 
   return v + before;
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkRows t) {
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_rows_kernel(const TopkRows t) {
   const int row = blockIdx.x;
   const int len = (t.len_mode == 0) ? t.len : (row % t.rows_per_group) + 1;
   const int forced = (t.forced_mode == 0) ? -1 : (t.forced_mode == 1) ? 0 : (row % t.rows_per_group);
   const float* sc = t.scores + (long long)row * t.row_stride;
   const int k = min(t.k, len);
-  __shared__ unsigned hist[256];
+  __shared__ unsigned hist[kTopkThreads / 32][256];  // one histogram per warp
   __shared__ unsigned long long wsum[32];
   __shared__ uint32_t sh_sel, sh_rem;
   auto key_of = [&](int j) -> uint32_t { return (j == forced) ? 0xFFFFFFFFu : order_key(sc[j]); };
@@ -305,30 +306,77 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkRows 
   // radix select of the k-th largest key, 8 bits at a time from the top
   uint32_t prefix = 0, pmask = 0, rem = (uint32_t)k;
   for (int shift = 24; shift >= 0 && k > 0; shift -= 8) {
-    for (int x = threadIdx.x; x < 256; x += blockDim.x) hist[x] = 0;
+    // long rows: one histogram per warp; short rows: one for the block
+    const int nh = (blockDim.x >= 1024) ? (blockDim.x >> 5) : 1;
+    unsigned* my_hist = hist[(blockDim.x >= 1024) ? (threadIdx.x >> 5) : 0];
+    for (int x = threadIdx.x; x < nh * 256; x += blockDim.x) hist[x >> 8][x & 255] = 0;
     __syncthreads();
-    for (int base = 0; base < len; base += blockDim.x) {
-      const int j = base + threadIdx.x;
-      uint32_t digit = 256;
-      if (j < len) {
-        const uint32_t key = key_of(j);
-        if ((key & pmask) == prefix) digit = (key >> shift) & 255u;
+    // each thread counts runs of equal digits in registers and adds a run
+    // when its digit changes
+    uint32_t last = 256;
+    unsigned run = 0;
+    // kTopkLoads independent coalesced loads per thread in flight per step
+    for (int base = 0; base < len; base += blockDim.x * kTopkLoads) {
+      uint32_t digit[kTopkLoads];
+#pragma unroll
+      for (int e = 0; e < kTopkLoads; ++e) {
+        const int j = base + e * blockDim.x + threadIdx.x;
+        digit[e] = 256;
+        if (j < len) {
+          const uint32_t key = key_of(j);
+          if ((key & pmask) == prefix) digit[e] = (key >> shift) & 255u;
+        }
       }
-      const unsigned same = __match_any_sync(0xFFFFFFFFu, digit);
-      if (digit < 256 && (threadIdx.x & 31) == (__ffs(same) - 1)) atomicAdd(&hist[digit], __popc(same));
+#pragma unroll
+      for (int e = 0; e < kTopkLoads; ++e) {
+        if (digit[e] != last) {
+          if (last < 256) atomicAdd(&my_hist[last], run);
+          last = digit[e];
+          run = 0;
+        }
+        ++run;
+      }
+    }
+    if (last < 256) atomicAdd(&my_hist[last], run);
+    __syncthreads();
+    // sum the warps' histograms into the first, in a fixed order
+    for (int x = threadIdx.x; x < 256 && nh > 1; x += blockDim.x) {
+      unsigned c = hist[0][x];
+      for (int w = 1; w < nh; ++w) c += hist[w][x];
+      hist[0][x] = c;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      uint32_t cum = 0, sel = 0;
-      for (int dgt = 255; dgt >= 0; --dgt) {
-        if (cum + hist[dgt] >= rem) {
-          sel = (uint32_t)dgt;
-          break;
-        }
-        cum += hist[dgt];
+    if (threadIdx.x < 32) {
+      // the digit holding the rem-th largest key: lane l owns digits
+      // 255 - 8l down to 248 - 8l; a scan over lanes finds the crossing
+      const int lane = threadIdx.x;
+      uint32_t h[8], sum = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        h[e] = hist[0][255 - 8 * lane - e];
+        sum += h[e];
       }
-      sh_sel = sel;
-      sh_rem = rem - cum;
+      uint32_t inc = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      const unsigned ball = __ballot_sync(0xFFFFFFFFu, inc >= rem);
+      const int owner = ball ? __ffs(ball) - 1 : 0;
+      if (lane == owner) {
+        uint32_t cum = inc - sum, sel = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (cum + h[e] >= rem) {
+            sel = (uint32_t)(255 - 8 * lane - e);
+            break;
+          }
+          cum += h[e];
+        }
+        sh_sel = sel;
+        sh_rem = rem - cum;
+      }
     }
     __syncthreads();
     prefix |= sh_sel << shift;
@@ -378,9 +426,212 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkRows 
   if (t.out_cnt && threadIdx.x == 0) t.out_cnt[row] = k;
 }
 
+// ---------------------------------------------- top-k of long rows, many CTAs
+// The same selection as topk_rows_kernel, for rows too long for one CTA: the
+// threshold key T is found by three radix passes (11, 11 and 10 bits) whose
+// histograms are gathered from (segment, row) CTAs into a per-row histogram
+// and resolved by one CTA per row; then every segment counts its keys above
+// and equal to T, and writes its selected indices at the offset given by the
+// counts of the segments before it (ascending order, lowest-index ties).
+// Per-row scratch: [0, 2048) histogram, [2048, 2051) prefix / mask / rem,
+// [2056, 2056 + 2 * 1024) per-segment (above, equal) counts.
+constexpr int kMsState = 2048;
+constexpr int kMsCounts = 2056;
+constexpr int kMsThreads = 512;
+
+struct TopkRowView {
+  const float* sc;
+  int len, forced, k;
+  __device__ TopkRowView(const TopkRows& t, int row) {
+    sc = t.scores + (long long)row * t.row_stride;
+    len = t.len;
+    forced = (t.forced_mode == 1) ? 0 : -1;
+    k = min(t.k, len);
+  }
+  __device__ uint32_t key(int j) const { return (j == forced) ? 0xFFFFFFFFu : order_key(sc[j]); }
+};
+
+__global__ void __launch_bounds__(256) topk_ms_init_kernel(const TopkRows t) {
+  uint32_t* ws = t.scratch + (size_t)blockIdx.x * kTopkScratchWords;
+  for (int x = threadIdx.x; x < kMsState; x += blockDim.x) ws[x] = 0;
+  if (threadIdx.x == 0) {
+    ws[kMsState] = 0;
+    ws[kMsState + 1] = 0;
+    ws[kMsState + 2] = (uint32_t)min(t.k, t.len);
+  }
+}
+
+template <int SHIFT, int BITS>
+__global__ void __launch_bounds__(kMsThreads) topk_ms_hist_kernel(const TopkRows t, int seg) {
+  constexpr int NB = 1 << BITS;
+  __shared__ unsigned h[NB];
+  const int row = blockIdx.y;
+  const TopkRowView r(t, row);
+  uint32_t* ws = t.scratch + (size_t)row * kTopkScratchWords;
+  const uint32_t prefix = ws[kMsState], pmask = ws[kMsState + 1];
+  for (int x = threadIdx.x; x < NB; x += blockDim.x) h[x] = 0;
+  __syncthreads();
+  const int j0 = blockIdx.x * seg, j1 = min(r.len, j0 + seg);
+  for (int base = j0; base < j1; base += blockDim.x * kTopkLoads) {
+    uint32_t kk[kTopkLoads];
+#pragma unroll
+    for (int e = 0; e < kTopkLoads; ++e) {
+      const int j = base + e * blockDim.x + threadIdx.x;
+      kk[e] = (j < j1) ? r.key(j) : 0u;
+    }
+#pragma unroll
+    for (int e = 0; e < kTopkLoads; ++e) {
+      const int j = base + e * blockDim.x + threadIdx.x;
+      if (j < j1 && (kk[e] & pmask) == prefix) atomicAdd(&h[(kk[e] >> SHIFT) & (NB - 1)], 1u);
+    }
+  }
+  __syncthreads();
+  for (int x = threadIdx.x; x < NB; x += blockDim.x)
+    if (h[x]) atomicAdd(&ws[x], h[x]);
+}
+
+// Resolves one pass: the digit holding the rem-th largest remaining key, and
+// clears the histogram for the next pass.
+template <int SHIFT, int BITS>
+__global__ void __launch_bounds__(1024) topk_ms_select_kernel(const TopkRows t) {
+  constexpr int NB = 1 << BITS;
+  constexpr int PER = NB / 1024;  // bins per thread, descending
+  __shared__ unsigned long long wsum[32];
+  uint32_t* ws = t.scratch + (size_t)blockIdx.x * kTopkScratchWords;
+  const uint32_t rem = ws[kMsState + 2];
+  uint32_t c[PER], sum = 0;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    c[e] = ws[NB - 1 - PER * threadIdx.x - e];
+    sum += c[e];
+  }
+  unsigned long long tot;
+  const unsigned long long inc = block_scan_u64(sum, wsum, tot);
+  const unsigned long long before = inc - sum;
+  if (before < rem && inc >= rem) {
+    uint32_t cum = (uint32_t)before, d = 0;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      if (cum + c[e] >= rem) {
+        d = (uint32_t)(NB - 1 - PER * threadIdx.x - e);
+        break;
+      }
+      cum += c[e];
+    }
+    ws[kMsState] |= d << SHIFT;
+    ws[kMsState + 1] |= (uint32_t)(NB - 1) << SHIFT;
+    ws[kMsState + 2] = rem - cum;
+  }
+  __syncthreads();
+  for (int x = threadIdx.x; x < NB; x += blockDim.x) ws[x] = 0;
+}
+
+// Keys above and equal to the threshold, per segment.
+__global__ void __launch_bounds__(kMsThreads) topk_ms_count_kernel(const TopkRows t, int seg) {
+  __shared__ unsigned long long wsum[32];
+  const int row = blockIdx.y;
+  const TopkRowView r(t, row);
+  uint32_t* ws = t.scratch + (size_t)row * kTopkScratchWords;
+  const uint32_t T = ws[kMsState];
+  const int j0 = blockIdx.x * seg, j1 = min(r.len, j0 + seg);
+  unsigned gt = 0, eq = 0;
+  for (int base = j0; base < j1; base += blockDim.x * kTopkLoads) {
+#pragma unroll
+    for (int e = 0; e < kTopkLoads; ++e) {
+      const int j = base + e * blockDim.x + threadIdx.x;
+      if (j < j1) {
+        const uint32_t kk = r.key(j);
+        gt += kk > T;
+        eq += kk == T;
+      }
+    }
+  }
+  unsigned long long tot;
+  block_scan_u64(((unsigned long long)gt << 32) | eq, wsum, tot);
+  if (threadIdx.x == 0) {
+    ws[kMsCounts + 2 * blockIdx.x] = (uint32_t)(tot >> 32);
+    ws[kMsCounts + 2 * blockIdx.x + 1] = (uint32_t)tot;
+  }
+}
+
+// Writes each segment's selected indices after those of the segments before it.
+__global__ void __launch_bounds__(kMsThreads) topk_ms_write_kernel(const TopkRows t, int seg) {
+  __shared__ unsigned long long wsum[32];
+  const int row = blockIdx.y, sgi = blockIdx.x;
+  const TopkRowView r(t, row);
+  const uint32_t* ws = t.scratch + (size_t)row * kTopkScratchWords;
+  const uint32_t T = ws[kMsState];
+  const unsigned long long need = ws[kMsState + 2];
+  unsigned long long pre = 0;
+  for (int s2 = threadIdx.x; s2 < sgi; s2 += blockDim.x)
+    pre += ((unsigned long long)ws[kMsCounts + 2 * s2] << 32) | ws[kMsCounts + 2 * s2 + 1];
+  unsigned long long tot;
+  block_scan_u64(pre, wsum, tot);
+  unsigned long long gt_before = tot >> 32, eq_before = tot & 0xFFFFFFFFull;
+  int32_t* out = t.out_idx + (long long)row * t.k;
+  const int j0 = sgi * seg, j1 = min(r.len, j0 + seg);
+  const int chunk = blockDim.x * kTopkItems;
+  for (int base = j0; base < j1; base += chunk) {
+    uint32_t keys[kTopkItems];
+    unsigned cgt = 0, ceq = 0;
+#pragma unroll
+    for (int e = 0; e < kTopkItems; ++e) {
+      const int j = base + threadIdx.x * kTopkItems + e;
+      const bool valid = j < j1;
+      keys[e] = valid ? r.key(j) : 0u;
+      cgt += (valid && keys[e] > T);
+      ceq += (valid && keys[e] == T);
+    }
+    unsigned long long ctot;
+    const unsigned long long inc = block_scan_u64(((unsigned long long)cgt << 32) | ceq, wsum, ctot);
+    const unsigned long long exc = inc - (((unsigned long long)cgt << 32) | ceq);
+    unsigned long long g = gt_before + (exc >> 32), q = eq_before + (exc & 0xFFFFFFFFull);
+#pragma unroll
+    for (int e = 0; e < kTopkItems; ++e) {
+      const int j = base + threadIdx.x * kTopkItems + e;
+      if (j < j1) {
+        if (keys[e] > T) {
+          out[g + min(q, need)] = j;
+          ++g;
+        } else if (keys[e] == T) {
+          if (q < need) out[g + q] = j;
+          ++q;
+        }
+      }
+    }
+    gt_before += ctot >> 32;
+    eq_before += ctot & 0xFFFFFFFFull;
+  }
+  if (sgi == 0) {
+    for (int x = r.k + threadIdx.x; x < t.k; x += blockDim.x) out[x] = -1;
+    if (t.out_cnt && threadIdx.x == 0) t.out_cnt[row] = r.k;
+  }
+}
+
+static cudaError_t topk_long_rows_launch(const TopkRows& t, cudaStream_t stream) {
+  const int seg = max(16384, (t.len + 1023) / 1024);
+  const int nseg = (t.len + seg - 1) / seg;
+  const dim3 g2(nseg, t.rows);
+  topk_ms_init_kernel<<<t.rows, 256, 0, stream>>>(t);
+  topk_ms_hist_kernel<21, 11><<<g2, kMsThreads, 0, stream>>>(t, seg);
+  topk_ms_select_kernel<21, 11><<<t.rows, 1024, 0, stream>>>(t);
+  topk_ms_hist_kernel<10, 11><<<g2, kMsThreads, 0, stream>>>(t, seg);
+  topk_ms_select_kernel<10, 11><<<t.rows, 1024, 0, stream>>>(t);
+  topk_ms_hist_kernel<0, 10><<<g2, kMsThreads, 0, stream>>>(t, seg);
+  topk_ms_select_kernel<0, 10><<<t.rows, 1024, 0, stream>>>(t);
+  topk_ms_count_kernel<<<g2, kMsThreads, 0, stream>>>(t, seg);
+  topk_ms_write_kernel<<<g2, kMsThreads, 0, stream>>>(t, seg);
+  return cudaGetLastError();
+}
+
 cudaError_t topk_rows_launch(const TopkRows& t, cudaStream_t stream) {
   if (t.rows <= 0) return cudaSuccess;
-  topk_rows_kernel<<<t.rows, kTopkThreads, 0, stream>>>(t);
+  if (t.len_mode == 0 && t.len > kTopkLongRow && t.scratch && t.forced_mode != 2)
+    return topk_long_rows_launch(t, stream);
+  // long rows (Vertical-Slash: one per head) take a whole SM each; short
+  // rows (Block-Sparse: one per query block) run several CTAs per SM
+  const int threads = (t.len > 32768) ? kTopkThreads : 256;
+  topk_rows_kernel<<<t.rows, threads, 0, stream>>>(t);
   return cudaGetLastError();
 }
 

@@ -81,7 +81,13 @@ struct TopkRows {
   int32_t* out_idx;      // [rows, k] ascending, -1 padded
   int32_t* out_cnt;      // [rows] or NULL
   DevStatus* status;
+  uint32_t* scratch;     // rows * kTopkScratchWords words for rows longer than kTopkLongRow, or NULL
 };
+// Rows longer than this (with len_mode 0) are split over many CTAs, given
+// topk_scratch_words(rows) words of scratch; shorter rows take one CTA each.
+constexpr int kTopkLongRow = 32768;
+constexpr int kTopkScratchWords = 2048 + 8 + 2 * 1024;
+inline size_t topk_scratch_words(int rows) { return (size_t)rows * kTopkScratchWords; }
 cudaError_t topk_rows_launch(const TopkRows& t, cudaStream_t stream);
 
 struct BsEstParams {

@@ -62,10 +62,23 @@ def make_plan(w: Workload, device="cuda") -> LayerPlan:
     return plan
 
 
-# kernels launched per layer: VS estimation 6 (two score passes, row combine,
-# slash combine, two top-k), VS index build 3, BS estimation 3 (pool, pooled
-# scores, top-k), and one attention launch per pattern
-LAUNCHES_PER_STEP = 6 + 3 + 1 + 3 + 1 + 1
+# rows longer than this take the many-CTA top-k (nine launches instead of one)
+TOPK_LONG_ROW = 32768
+
+
+def launches_per_step(plan: LayerPlan) -> int:
+    """Kernels one run_layer call launches: VS estimation (two score passes,
+    row combine, slash combine, two top-k), VS index build 3, BS estimation
+    3 (pool, pooled scores, top-k), and one attention launch per pattern."""
+    n = 0
+    if plan.vs_heads is not None:
+        topk = 9 if plan.w.N > TOPK_LONG_ROW else 1
+        n += 4 + 2 * topk + 3 + 1
+    if plan.bs_heads is not None:
+        n += 3 + 1
+    if plan.a_heads is not None:
+        n += 1
+    return n
 
 
 def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None, marks=None):

@@ -224,3 +224,22 @@ def test_minimum_size_one_tile(d):
     _check_attn(o, lse, qn, kn, vn, [0, 1], w, lambda hi, h: (lambda r: orc.mask_ashape(r, w.N, 16, 32)))
     o, lse = minf.minf_dense_attn(q, k, v)
     _check_attn(o, lse, qn, kn, vn, [0, 1], w, lambda hi, h: (lambda r: orc.mask_dense(r, w.N)))
+
+
+@pytest.mark.parametrize("N,k_v,k_s", [(65536, 1000, 3000), (131072, 2000, 6000)])
+def test_vs_estimation_long_rows(N, k_v, k_s):
+    """Rows longer than 32K take the many-CTA top-k (several segments per row)."""
+    w = wl.small(Hq=2, Hkv=1, N=N, d=64, seed=35, k_v=k_v, k_s=k_s)
+    q, k, v, qn, kn, vn = _inputs(w)
+    sc = orc.default_scale(w.d)
+    ws = minf.workspace(minf.OP_ESTIMATE_VS, minf.shape_of(q, k), 2)
+    v_idx, s_idx, vs, ss = minf.minf_estimate_vs(q, k, [0, 1], k_v, k_s, return_scores=True, ws=ws)
+    assert minf.minf_get_device_status(ws) == 0
+    gv, gs = v_idx[0].cpu().numpy(), s_idx[0].cpu().numpy()
+    for h in range(2):
+        rv, rs = orc.vs_estimate(qn[h][N - 64:], kn[0], sc)
+        np.testing.assert_allclose(vs[0, h].cpu().numpy(), rv, rtol=1e-4, atol=1e-7)
+        ov, os_ = orc.vs_select(rv, rs, k_v, k_s)
+        assert np.all(np.diff(gv[h]) > 0) and np.all(np.diff(gs[h]) > 0)
+        check_index_set(gv[h], ov, rv, what=f"vertical h{h}")
+        check_index_set(gs[h], os_, rs, forced=0, what=f"slash h{h}")
