@@ -19,6 +19,10 @@ page and the abstract):
 * attention computed only over the estimated indices (summary, "Summary",
   stage 3).
 
+Besides the band reading of a slash (``mask_vs``), ``mask_vs_exact`` and
+``vs_exact_index`` give the element-exact variant, where a slash is its
+diagonal only.
+
 The pages fix nothing finer.  The readings taken where they are silent
 (last 64 queries; natural-exp softmax with scale 1/sqrt(d) before the column
 and diagonal sums; forced slash offset 0 and forced diagonal block; ties to
@@ -286,6 +290,39 @@ def mask_vs(rows, N: int, v_idx, s_idx, block: int = 64) -> np.ndarray:
         n_in = np.searchsorted(s, u + block - 1, side="right") - np.searchsorted(s, u, side="left")
         out[r] = (j <= i) & (vert | (n_in > 0))
     return out
+
+
+def mask_vs_exact(rows, N: int, v_idx, s_idx) -> np.ndarray:
+    """Element-exact Vertical-Slash: causal and (j in V or i - j in S).
+
+    The slashes are the selected diagonals themselves, element by element,
+    instead of the 64-key bands they sweep through a 64-row query block
+    (:func:`mask_vs`); the exact set is contained in the band set.
+    """
+    rows = np.asarray(rows)
+    vert = np.zeros(N, bool)
+    vert[np.asarray(v_idx, np.int64)] = True
+    diag = np.zeros(N, bool)
+    diag[np.asarray(s_idx, np.int64)] = True
+    j = np.arange(N)
+    out = np.zeros((rows.size, N), bool)
+    for r, i in enumerate(rows):
+        o = i - j
+        causal = o >= 0
+        out[r] = causal & (vert | np.where(causal, diag[np.clip(o, 0, N - 1)], False))
+    return out
+
+
+def vs_exact_index(v_idx, s_idx, N: int, tile: int = 128):
+    """Index of the element-exact variant for query tiles of ``tile`` rows:
+    the offsets merged at gap <= tile (each group's diagonals sweep the key
+    range [R - b_g, R + tile - 1 - a_g] of the tile starting at row R), and
+    per tile the verticals outside every such range (they are the only keys
+    of V that the ranges do not already hold).  Returns (groups, vcnt, vidx)
+    as :func:`vs_build_index` with blocks of ``tile`` rows."""
+    groups = vs_groups(s_idx, tile)
+    vcnt, vidx = vs_block_verticals(v_idx, groups, N, tile)
+    return groups, vcnt, vidx
 
 
 def mask_bs(rows, N: int, blk_idx, blk_cnt, block: int = 64) -> np.ndarray:

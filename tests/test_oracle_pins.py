@@ -55,6 +55,15 @@ def test_golden_vs_mask():
     assert np.array_equal(got, _to_mask(rows, N))
 
 
+def test_golden_vs_exact_mask():
+    p, rows = _golden_cases()["vs_exact"]
+    N = int(p["N"])
+    V = [int(x) for x in p["V"].split(",")]
+    S = [int(x) for x in p["S"].split(",")]
+    got = orc.mask_vs_exact(np.arange(N), N, V, S)
+    assert np.array_equal(got, _to_mask(rows, N))
+
+
 def test_golden_bs_mask():
     p, rows = _golden_cases()["bs"]
     N, blk = int(p["N"]), int(p["block"])
@@ -341,3 +350,70 @@ def test_vs_block_verticals_direct_intervals():
         ref = [j for j in V if j <= r0 + 63 and
                not any(r0 - bg <= j <= r0 + 63 - ag for ag, bg in groups)]
         assert vidx[b, : vcnt[b]].tolist() == ref
+
+
+# ------------------------------------------------ element-exact VS variant
+
+def test_vs_exact_mask_bruteforce_loops():
+    rng = np.random.default_rng(40)
+    N = 48
+    S = sorted(set([0] + rng.choice(N, 9, replace=False).tolist()))
+    V = sorted(set(rng.choice(N, 6, replace=False).tolist()))
+    got = orc.mask_vs_exact(np.arange(N), N, V, S)
+    for i in range(N):
+        for j in range(N):
+            assert got[i, j] == (j <= i and (j in V or (i - j) in S)), (i, j)
+
+
+def test_vs_exact_mask_closed_forms():
+    N = 200
+    i, j = np.meshgrid(np.arange(N), np.arange(N), indexing="ij")
+    assert np.array_equal(orc.mask_vs_exact(np.arange(N), N, [], np.arange(N)), j <= i)
+    assert np.array_equal(orc.mask_vs_exact(np.arange(N), N, [], [0]), i == j)
+    assert np.array_equal(orc.mask_vs_exact(np.arange(N), N, [7], [0]), (i == j) | ((j == 7) & (i >= 7)))
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_vs_exact_mask_within_band_mask(seed):
+    """The exact diagonals are a subset of the bands they sweep (the band
+    reading is a superset)."""
+    rng = np.random.default_rng(50 + seed)
+    N = 64 * 9
+    S = np.unique(np.concatenate([[0], rng.choice(N, 30, replace=False)]))
+    V = np.unique(rng.choice(N, 20, replace=False))
+    ex = orc.mask_vs_exact(np.arange(N), N, V, S)
+    band = orc.mask_vs(np.arange(N), N, V, S)
+    assert not (ex & ~band).any()
+    assert ex.sum() < band.sum()
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_vs_exact_index_reproduces_mask(seed):
+    """Per 128-row query tile: the key ranges of the offset groups (gap <= 128),
+    masked element by element with (i - j in S or j in V), plus the tile's
+    vertical list, give exactly the exact mask; the list never repeats a key
+    of the ranges."""
+    rng = np.random.default_rng(60 + seed)
+    N = 128 * 6
+    S = np.unique(np.concatenate([[0], rng.choice(N, 40 + 10 * seed, replace=False)]))
+    V = np.unique(rng.choice(N, 50, replace=False))
+    groups, vcnt, vidx = orc.vs_exact_index(V, S, N)
+    sset, vset = set(S.tolist()), set(V.tolist())
+    ref = orc.mask_vs_exact(np.arange(N), N, V, S)
+    got = np.zeros((N, N), bool)
+    for t in range(N // 128):
+        R = 128 * t
+        rng_keys = set()
+        for a_g, b_g in groups:
+            rng_keys.update(range(max(0, R - b_g), max(0, R + 128 - a_g)))
+        lst = vidx[t, : vcnt[t]].tolist()
+        assert not (set(lst) & rng_keys)
+        assert lst == sorted(lst)
+        for i in range(R, R + 128):
+            for j in rng_keys:
+                if j <= i and ((i - j) in sset or j in vset):
+                    got[i, j] = True
+            for j in lst:
+                if j <= i:
+                    got[i, j] = True
+    assert np.array_equal(got, ref)
