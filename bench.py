@@ -362,6 +362,39 @@ def run_ours(args, dist, rank, world, local):
         dense_ms = d0.elapsed_time(d1) * w.Hq
         del od
 
+    # element-exact Vertical-Slash variant on the layer's VS heads and sets
+    # (outside the timed step: index build and attention, CUDA events)
+    vs_exact = None
+    if rank == 0 and not args.no_exact and plan.vs_heads is not None:
+        b = plan.bufs
+        ws_x = minf.workspace(minf.OP_SPARSE_ATTN_VS_EXACT, plan.shape, plan.vs_heads.numel(), device=dev)
+        ws_xi = minf.workspace(minf.OP_BUILD_INDEX_EXACT, plan.shape, plan.vs_heads.numel(), device=dev)
+        xi = minf.minf_build_index_exact(plan.shape, b["v_idx"], b["s_idx"], ws=ws_xi)
+        ox = o  # the timed steps are done; reuse the output buffer
+        ws_x.zero_()
+        minf.minf_sparse_attn_vs_exact(q, k, v, plan.vs_heads, xi, o=ox, want_lse=False, ws=ws_x)
+        torch.cuda.synchronize()
+        if minf.minf_get_device_status(ws_xi) or minf.minf_get_device_status(ws_x):
+            raise RuntimeError("exact variant reported a device error")
+        x_tiles, x_nnz = _counters(ws_x)
+        xe = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        xe[0].record(stream)
+        minf.minf_build_index_exact(plan.shape, b["v_idx"], b["s_idx"], index=xi, ws=ws_xi)
+        xe[1].record(stream)
+        for _ in range(2):
+            minf.minf_sparse_attn_vs_exact(q, k, v, plan.vs_heads, xi, o=ox, want_lse=False, ws=ws_x)
+        xe[2].record(stream)
+        torch.cuda.synchronize()
+        x_ms = xe[1].elapsed_time(xe[2]) / 2
+        vs_exact = {
+            "attn_ms": round(x_ms, 3), "index_ms": round(xe[0].elapsed_time(xe[1]), 3),
+            "executed_tflop": tile_flops * x_tiles / 1e12, "useful_tflop": 4.0 * w.d * x_nnz / 1e12,
+            "executed_tflops": tile_flops * x_tiles / (x_ms * 1e-3) / 1e12,
+            "useful_tflops": 4.0 * w.d * x_nnz / (x_ms * 1e-3) / 1e12,
+            "band_useful_tflop": 4.0 * w.d * cnt["ws_vs_attn"][1] / 1e12,
+        }
+        del xi
+
     if rank != 0:
         return
     peaks, src = _peaks()
@@ -402,6 +435,7 @@ def run_ours(args, dist, rank, world, local):
         "gpu_launches": layer.launches_per_step(plan) * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
+        "vs_exact": ({**vs_exact, "frac": vs_exact["executed_tflops"] / peak} if vs_exact else None),
     }
     print(json.dumps(line), flush=True)
 
@@ -441,6 +475,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense baseline")
+    ap.add_argument("--no-exact", action="store_true", help="skip the element-exact VS variant")
     ap.add_argument("--kernel", choices=["dense", "vs"], default=None,
                     help="run only this attention kernel on a small case (for profiling)")
     ap.add_argument("--N", type=int, default=262144, help="tokens of the --kernel case")

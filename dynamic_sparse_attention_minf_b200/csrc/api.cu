@@ -159,6 +159,8 @@ minf_status attn_launch(int pol, const minf_shape* s, const AttnParams& p, void*
 extern "C" {
 
 size_t minf_vs_wmap_words(int N) { return N > 0 ? (size_t)(N + 64) / 32 + 2 : 0; }
+size_t minf_vs_bits_words(int N) { return N > 0 ? (size_t)N / 32 + 8 : 0; }
+size_t minf_vs_twmap_words(int N) { return N > 0 ? (size_t)(N + 128) / 32 + 2 : 0; }
 
 size_t minf_workspace_size(int op, const minf_shape* s, int nh, int k_v, int k_s, int k_b) {
   (void)k_v;
@@ -171,6 +173,8 @@ size_t minf_workspace_size(int op, const minf_shape* s, int nh, int k_v, int k_s
     case MINF_OP_ESTIMATE_BS:
       return plan_bs_est(s, nh, nullptr, nullptr);
     case MINF_OP_BUILD_INDEX:
+    case MINF_OP_BUILD_INDEX_EXACT:
+    case MINF_OP_SPARSE_ATTN_VS_EXACT:
     case MINF_OP_SPARSE_ATTN_VS:
     case MINF_OP_SPARSE_ATTN_BS:
     case MINF_OP_ATTN_ASHAPE:
@@ -309,6 +313,53 @@ minf_status minf_build_index(const minf_shape* s, int nh, const int32_t* v_idx, 
   p.idx = *idx;
   p.status = reinterpret_cast<DevStatus*>(ws);
   return cuda_status(vs_index_launch(p, (cudaStream_t)stream));
+}
+
+minf_status minf_build_index_exact(const minf_shape* s, int nh, const int32_t* v_idx, int k_v,
+                                   const int32_t* s_idx, int k_s, const minf_vs_exact_index* idx, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  minf_status st = check_shape(s);
+  if (st != MINF_OK) return st;
+  if (!v_idx || !s_idx || !idx || !ws || nh < 1) return MINF_ERR_INVALID_ARG;
+  if (!idx->tgrp || !idx->tgrp_cnt || !idx->sbits || !idx->vbits || !idx->twmap || !idx->vcnt || !idx->vidx)
+    return MINF_ERR_INVALID_ARG;
+  if (k_v < 1 || k_s < 1 || k_v > s->N || k_s > s->N) return MINF_ERR_INVALID_ARG;
+  if (ws_bytes < kStatusBytes) return MINF_ERR_WORKSPACE_TOO_SMALL;
+  VsIndexParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.v_idx = v_idx;
+  p.s_idx = s_idx;
+  p.nh = nh;
+  p.B = s->B;
+  p.N = s->N;
+  p.k_v = k_v;
+  p.k_s = k_s;
+  p.status = reinterpret_cast<DevStatus*>(ws);
+  return cuda_status(vs_exact_index_launch(p, *idx, (int)minf_vs_bits_words(s->N), (int)minf_vs_twmap_words(s->N),
+                                           (cudaStream_t)stream));
+}
+
+minf_status minf_sparse_attn_vs_exact(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K,
+                                      const minf_bf16* V, const int32_t* heads, int nh,
+                                      const minf_vs_exact_index* idx, int k_v, int k_s, minf_bf16* O, float* lse,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  minf_status st = attn_common(POL_VS_EXACT, s, Q, K, V, heads, nh, O, lse, ws, ws_bytes, stream, p);
+  if (st != MINF_OK) return st;
+  if (!idx || !idx->tgrp || !idx->tgrp_cnt || !idx->sbits || !idx->vbits || !idx->vcnt || !idx->vidx)
+    return MINF_ERR_INVALID_ARG;
+  if (k_v < 1 || k_s < 1 || k_v > s->N || k_s > s->N) return MINF_ERR_INVALID_ARG;
+  p.tgrp = idx->tgrp;
+  p.tgrp_cnt = idx->tgrp_cnt;
+  p.sbits = idx->sbits;
+  p.vbits = idx->vbits;
+  p.bits_words = (int)minf_vs_bits_words(s->N);
+  p.vcnt = idx->vcnt;
+  p.vidx = idx->vidx;
+  p.k_s = k_s;
+  p.k_v = k_v;
+  return attn_launch(POL_VS_EXACT, s, p, stream);
 }
 
 minf_status minf_sparse_attn_vs(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,

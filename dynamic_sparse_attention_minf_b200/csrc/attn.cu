@@ -33,7 +33,7 @@
 namespace minf {
 
 enum { KIND_END = 0, KIND_RANGE = 1, KIND_GATHER = 2 };
-enum { F_MASK = 1, F_CAUSAL = 2, F_ASHAPE = 4 };
+enum { F_MASK = 1, F_CAUSAL = 2, F_ASHAPE = 4, F_EXACT = 8 };
 
 struct TileDesc {
   int kind;
@@ -86,6 +86,31 @@ __device__ __forceinline__ uint32_t wmap_window(const uint32_t* W, int p) {
 }
 __device__ __forceinline__ uint32_t wmap_bit(const uint32_t* W, int x) {
   return (__ldg(W + (x >> 5)) >> (x & 31)) & 1u;
+}
+
+// Bits p .. p + 63 of a bitmap as one 64-bit value, bit k = bit p + k (bits
+// below 0 read as zero), from the three words starting at word max(p, 0) / 32
+// (loaded separately, so that the loads can be issued early).
+struct Window64 {
+  uint32_t w0, w1, w2;
+  int p;
+  __device__ __forceinline__ void load(const uint32_t* W, int p_) {
+    p = p_;
+    const int wi = max(p, 0) >> 5;
+    w0 = __ldg(W + wi);
+    w1 = __ldg(W + wi + 1);
+    w2 = __ldg(W + wi + 2);
+  }
+  __device__ __forceinline__ uint64_t bits() const {
+    if (p <= -64) return 0ull;
+    const int sh = max(p, 0) & 31;
+    uint64_t v = ((uint64_t)__funnelshift_r(w1, w2, sh) << 32) | __funnelshift_r(w0, w1, sh);
+    if (p < 0) v <<= -p;
+    return v;
+  }
+};
+__device__ __forceinline__ uint64_t brev64(uint64_t x) {
+  return ((uint64_t)__brev((uint32_t)x) << 32) | __brev((uint32_t)(x >> 32));
 }
 
 // A wait whose outcome is the same for every lane of the warp (the TMEM
@@ -364,22 +389,21 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi
     }
   } else if (POL == POL_ASHAPE) {
     const int lloc = max(0, R - p.n_local + 1);
-    int lo[2], hi_[2], n_iv = 0;
-    if (p.n_sink >= lloc) {
-      lo[0] = 0; hi_[0] = R + 127; n_iv = 1;
-    } else {
-      if (p.n_sink > 0) { lo[n_iv] = 0; hi_[n_iv] = p.n_sink - 1; ++n_iv; }
-      lo[n_iv] = lloc; hi_[n_iv] = R + 127; ++n_iv;
-    }
     const int far_edge = R + 127 - p.n_local;   // keys <= this may leave some row's window
-    for (int v = 0; v < n_iv; ++v) {
-      for (int j0 = lo[v]; j0 <= hi_[v] && P.ok; j0 += 128) {
-        const int cnt = min(128, hi_[v] - j0 + 1);
+    auto interval = [&](int lo, int hi_) {
+      for (int j0 = lo; j0 <= hi_ && P.ok; j0 += 128) {
+        const int cnt = min(128, hi_ - j0 + 1);
         const uint32_t word = (lane < 8) ? count_mask(cnt, lane & 3) : 0xFFFFFFFFu;
         int flags = (j0 + cnt - 1 > R) ? F_CAUSAL : 0;
         if (max(j0, p.n_sink) <= min(j0 + cnt - 1, far_edge)) flags |= F_ASHAPE;
         P.emit_range(j0, j0 + 64, word, flags);
       }
+    };
+    if (p.n_sink >= lloc) {
+      interval(0, R + 127);  // sinks and window touch: one interval
+    } else {
+      if (p.n_sink > 0) interval(0, p.n_sink - 1);
+      interval(lloc, R + 127);
     }
   } else if (POL == POL_VS) {
     const size_t hrow = (size_t)b * p.nh + hi;
@@ -481,6 +505,51 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi
       if (j < 0 || j > R + 63) { if (idx < c0) report(P.st, MINF_ERR_DEVICE_BOUNDS, 21); j = 0; }
       const bool keep = (idx < c0) && wmap_bit(W, R + 127 - j);
       P.append(keep, j, 1u, n_staged);
+    }
+    if (n_staged > 0 && P.ok) P.emit_gather(n_staged);
+  } else if (POL == POL_VS_EXACT) {
+    // The same key ranges as the band variant at 128-row granularity (one per
+    // offset group of gap 128), masked element by element by the softmax from
+    // the offset and key bitmaps; then the tile's own vertical list.
+    const size_t hrow = (size_t)b * p.nh + hi;
+    const int* tg = p.tgrp + hrow * p.k_s * 2;
+    const int G = p.tgrp_cnt[hrow];
+    int top = 0;
+    {
+      int lo = 0, hi2 = G;
+      while (lo < hi2) {
+        const int mid = (lo + hi2) >> 1;
+        if (__ldg(tg + 2 * mid) <= R + 127) lo = mid + 1; else hi2 = mid;
+      }
+      top = lo - 1;
+    }
+    for (int base = top; base >= 0 && P.ok; base -= 32) {
+      const int gl = base - lane;
+      int lo_l = 0, hi_l = -1;
+      if (gl >= 0) {
+        hi_l = min(R + 127 - __ldg(tg + 2 * gl), p.N - 1);
+        lo_l = max(0, R - __ldg(tg + 2 * gl + 1));
+      }
+      const int nbatch = min(32, base + 1);
+      for (int k = 0; k < nbatch && P.ok; ++k) {
+        const int lo_key = __shfl_sync(0xFFFFFFFFu, lo_l, k);
+        const int hi_key = __shfl_sync(0xFFFFFFFFu, hi_l, k);
+        for (int j0 = lo_key; j0 <= hi_key && P.ok; j0 += 128) {
+          const int cnt = min(128, hi_key - j0 + 1);
+          const uint32_t word = (lane < 8) ? count_mask(cnt, lane & 3) : 0xFFFFFFFFu;
+          P.emit_range(j0, j0 + 64, word, F_EXACT | ((j0 + cnt - 1 > R) ? F_CAUSAL : 0));
+        }
+      }
+    }
+    const int nt = p.N / 128;
+    const int* vl = p.vidx + (hrow * nt + qt) * (size_t)p.k_v;
+    const int c = min(p.vcnt[hrow * nt + qt], p.k_v);
+    int n_staged = 0;
+    for (int base = 0; base < c && P.ok; base += 32) {
+      const int idx = base + lane;
+      int j = (idx < c) ? vl[idx] : 0;
+      if (j < 0 || j > R + 127) { if (idx < c) report(P.st, MINF_ERR_DEVICE_BOUNDS, 24); j = 0; }
+      P.append(idx < c, j, (j <= R + 63 ? 1u : 0u) | 2u, n_staged);
     }
     if (n_staged > 0 && P.ok) P.emit_gather(n_staged);
   } else if (POL == POL_BS) {
@@ -750,6 +819,16 @@ __global__ void __launch_bounds__(320, 1)
       const TileDesc& dd = desc[st];
       const int kind = dd.kind;
       if (kind == KIND_END) break;
+      // element-exact tiles: the bitmap words of this row's window are
+      // requested before waiting for the scores
+      Window64 xs, xv;
+      const bool exact = POL == POL_VS_EXACT && (dd.flags & F_EXACT);
+      if (exact) {
+        const size_t hb = ((size_t)b * p.nh + hi) * p.bits_words;
+        const int jw = dd.j0[wg];
+        xs.load(p.sbits + hb, i - jw - 63);
+        xv.load(p.vbits + hb, jw);
+      }
       if (!warp_wait(&s_full[t & 1], (t >> 1) & 1, abort, p.status, 11)) break;
       tc_fence_after();
       const int flags = dd.flags;
@@ -763,6 +842,13 @@ __global__ void __launch_bounds__(320, 1)
         const uint2 m2 = *reinterpret_cast<const uint2*>(&dd.mask[half][2 * wg]);
         mw[0] = m2.x;
         mw[1] = m2.y;
+      }
+      if (exact) {
+        // bit c: (i - j in S) or (j in V) for key j = j0 + c; these words
+        // differ between rows, so the chunk tests below are per thread here
+        const uint64_t em = brev64(xs.bits()) | xv.bits();
+        mw[0] &= (uint32_t)em;
+        mw[1] &= (uint32_t)(em >> 32);
       }
       uint32_t sr[2][32];
       tmem_ld32(scol, sr[0]);
@@ -781,7 +867,7 @@ __global__ void __launch_bounds__(320, 1)
             if (!((mw[c2] >> e) & 1u)) s[c2 * 32 + e] = -INFINITY;
         }
       }
-      if (flags & (F_CAUSAL | F_ASHAPE)) {
+      if (flags & (F_CAUSAL | F_ASHAPE | F_EXACT)) {
         const bool causal = flags & F_CAUSAL;
         const bool ash = flags & F_ASHAPE;
         if (kind == KIND_RANGE) {
@@ -979,6 +1065,8 @@ cudaError_t attn_dispatch(int d, int pol, const CUtensorMap& tq, const CUtensorM
   MINF_CASE(128, POL_ASHAPE)
   MINF_CASE(128, POL_VS)
   MINF_CASE(128, POL_BS)
+  MINF_CASE(64, POL_VS_EXACT)
+  MINF_CASE(128, POL_VS_EXACT)
 #undef MINF_CASE
   return cudaErrorInvalidValue;
 }

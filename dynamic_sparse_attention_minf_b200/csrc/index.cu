@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(1024) vs_groups_kernel(const VsIndexParams p) 
     const int o = s[x];
     if (o < 0 || o >= p.N || (x > 0 && s[x - 1] >= o)) report(p.status, MINF_ERR_DEVICE_BOUNDS, 51);
   }
-  int32_t* grp = p.idx.grp + bh * p.k_s * 2;
+  int32_t* grp = p.idx.grp ? p.idx.grp + bh * p.k_s * 2 : nullptr;  // null: tile groups only
   int32_t* tgrp = p.idx.tgrp + bh * p.k_s * 2;
   int run_g = 0, run_t = 0;
   for (int base = 0; base < p.k_s; base += blockDim.x) {
@@ -75,28 +75,31 @@ __global__ void __launch_bounds__(1024) vs_groups_kernel(const VsIndexParams p) 
     // group index of element x = (#starts up to and including x) - 1
     const int gi = run_g + eg + (start_g ? 1 : 0) - 1;
     const int ti = run_t + et + (start_t ? 1 : 0) - 1;
-    if (start_g) grp[2 * gi] = o;
-    if (end_g) grp[2 * gi + 1] = o;
+    if (grp && start_g) grp[2 * gi] = o;
+    if (grp && end_g) grp[2 * gi + 1] = o;
     if (start_t) tgrp[2 * ti] = o;
     if (end_t) tgrp[2 * ti + 1] = o;
     run_g += tot_g;
     run_t += tot_t;
   }
   if (threadIdx.x == 0) {
-    p.idx.grp_cnt[bh] = run_g;
+    if (p.idx.grp_cnt) p.idx.grp_cnt[bh] = run_g;
     p.idx.tgrp_cnt[bh] = run_t;
   }
 }
 
-// One thread per bitmap word.
-__global__ void __launch_bounds__(256) vs_wmap_kernel(const VsIndexParams p) {
+// One thread per bitmap word: bit x set iff x - (BLK - 1) lies in some
+// [a_g - (BLK - 1), b_g] of the given groups (the groups of gap BLK).
+template <int BLK>
+__global__ void __launch_bounds__(256) vs_wmap_kernel(const VsIndexParams p, const int32_t* grps,
+                                                      const int32_t* gcnt, uint32_t* wmap, int words) {
   const int w = blockIdx.x * 256 + threadIdx.x;
   const int hi = blockIdx.y, b = blockIdx.z;
-  if (w >= p.wmap_words) return;
+  if (w >= words) return;
   const size_t bh = (size_t)b * p.nh + hi;
-  const int* grp = p.idx.grp + bh * p.k_s * 2;
-  const int G = p.idx.grp_cnt[bh];
-  const int u_lo = 32 * w - 63, u_hi = u_lo + 31;
+  const int* grp = grps + bh * p.k_s * 2;
+  const int G = gcnt[bh];
+  const int u_lo = 32 * w - (BLK - 1), u_hi = u_lo + 31;
   // first group with b_g >= u_lo
   int lo = 0, hi2 = G;
   while (lo < hi2) {
@@ -105,7 +108,7 @@ __global__ void __launch_bounds__(256) vs_wmap_kernel(const VsIndexParams p) {
   }
   uint32_t word = 0;
   for (int g = lo; g < G; ++g) {
-    const int a = grp[2 * g] - 63, bb = grp[2 * g + 1];
+    const int a = grp[2 * g] - (BLK - 1), bb = grp[2 * g + 1];
     if (a > u_hi) break;
     const int s0 = max(a, u_lo) - u_lo, s1 = min(bb, u_hi) - u_lo;
     if (s0 <= s1) {
@@ -114,29 +117,32 @@ __global__ void __launch_bounds__(256) vs_wmap_kernel(const VsIndexParams p) {
       word |= m;
     }
   }
-  p.idx.wmap[bh * p.wmap_words + w] = word;
+  wmap[bh * words + w] = word;
 }
 
-// One warp per 64-row query block.
-__global__ void __launch_bounds__(256) vs_vlist_kernel(const VsIndexParams p) {
+// One warp per BLK-row query block: the ascending vertical columns j <= the
+// block's last row whose bit (r0 - j + BLK - 1) of the group bitmap is clear.
+template <int BLK>
+__global__ void __launch_bounds__(256) vs_vlist_kernel(const VsIndexParams p, const uint32_t* wmap, int words,
+                                                       int32_t* vcnt, int32_t* vidx) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nb = p.N / 64;
+  const int nb = p.N / BLK;
   const int qb = blockIdx.x * 8 + warp;
   const int hi = blockIdx.y, b = blockIdx.z;
   if (qb >= nb) return;
   const size_t bh = (size_t)b * p.nh + hi;
   const int* v = p.v_idx + bh * p.k_v;
-  const uint32_t* W = p.idx.wmap + bh * p.wmap_words;
-  int32_t* out = p.idx.vidx + (bh * nb + qb) * (size_t)p.k_v;
-  const int r0 = qb * 64;
+  const uint32_t* W = wmap + bh * words;
+  int32_t* out = vidx + (bh * nb + qb) * (size_t)p.k_v;
+  const int r0 = qb * BLK;
   int n = 0;
   for (int base = 0; base < p.k_v; base += 32) {
     const int x = base + lane;
     const int j = (x < p.k_v) ? v[x] : 0x7FFFFFFF;
-    const bool inr = (j >= 0) && (j <= r0 + 63);
+    const bool inr = (j >= 0) && (j <= r0 + BLK - 1);
     bool keep = false;
     if (inr) {
-      const int bit = r0 - j + 63;
+      const int bit = r0 - j + BLK - 1;
       keep = !((__ldg(W + (bit >> 5)) >> (bit & 31)) & 1u);
     }
     const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
@@ -144,14 +150,54 @@ __global__ void __launch_bounds__(256) vs_vlist_kernel(const VsIndexParams p) {
     n += __popc(bal);
     if (!__all_sync(0xFFFFFFFFu, inr || x >= p.k_v)) break;  // list is ascending
   }
-  if (lane == 0) p.idx.vcnt[bh * nb + qb] = n;
+  if (lane == 0) vcnt[bh * nb + qb] = n;
+}
+
+// One thread per word of the offset and key bitmaps: bit o of sbits set iff
+// o is in S, bit j of vbits iff j is in V (both lists ascending).
+__global__ void __launch_bounds__(256) vs_bits_kernel(const VsIndexParams p, uint32_t* sbits, uint32_t* vbits,
+                                                      int words) {
+  const int w = blockIdx.x * 256 + threadIdx.x;
+  const int hi = blockIdx.y, b = blockIdx.z;
+  if (w >= words) return;
+  const size_t bh = (size_t)b * p.nh + hi;
+  auto word_of = [&](const int* lst, int n) -> uint32_t {
+    int lo = 0, hi2 = n;  // first element >= 32 w
+    while (lo < hi2) {
+      const int mid = (lo + hi2) >> 1;
+      if (lst[mid] < 32 * w) lo = mid + 1; else hi2 = mid;
+    }
+    uint32_t word = 0;
+    for (int x = lo; x < n && lst[x] < 32 * w + 32; ++x) word |= 1u << (lst[x] - 32 * w);
+    return word;
+  };
+  sbits[bh * words + w] = word_of(p.s_idx + bh * p.k_s, p.k_s);
+  vbits[bh * words + w] = word_of(p.v_idx + bh * p.k_v, p.k_v);
 }
 
 cudaError_t vs_index_launch(const VsIndexParams& p, cudaStream_t stream) {
   vs_groups_kernel<<<dim3(p.nh, p.B), 1024, 0, stream>>>(p);
-  vs_wmap_kernel<<<dim3((p.wmap_words + 255) / 256, p.nh, p.B), 256, 0, stream>>>(p);
+  vs_wmap_kernel<64><<<dim3((p.wmap_words + 255) / 256, p.nh, p.B), 256, 0, stream>>>(
+      p, p.idx.grp, p.idx.grp_cnt, p.idx.wmap, p.wmap_words);
   const int nb = p.N / 64;
-  vs_vlist_kernel<<<dim3((nb + 7) / 8, p.nh, p.B), 256, 0, stream>>>(p);
+  vs_vlist_kernel<64><<<dim3((nb + 7) / 8, p.nh, p.B), 256, 0, stream>>>(p, p.idx.wmap, p.wmap_words, p.idx.vcnt,
+                                                                        p.idx.vidx);
+  return cudaGetLastError();
+}
+
+cudaError_t vs_exact_index_launch(const VsIndexParams& p, const minf_vs_exact_index& x, int bits_words,
+                                  int twmap_words, cudaStream_t stream) {
+  VsIndexParams q = p;  // tile groups only
+  q.idx.grp = nullptr;
+  q.idx.grp_cnt = nullptr;
+  q.idx.tgrp = x.tgrp;
+  q.idx.tgrp_cnt = x.tgrp_cnt;
+  vs_groups_kernel<<<dim3(q.nh, q.B), 1024, 0, stream>>>(q);
+  vs_bits_kernel<<<dim3((bits_words + 255) / 256, q.nh, q.B), 256, 0, stream>>>(q, x.sbits, x.vbits, bits_words);
+  vs_wmap_kernel<128><<<dim3((twmap_words + 255) / 256, q.nh, q.B), 256, 0, stream>>>(q, x.tgrp, x.tgrp_cnt,
+                                                                                     x.twmap, twmap_words);
+  const int nt = q.N / 128;
+  vs_vlist_kernel<128><<<dim3((nt + 7) / 8, q.nh, q.B), 256, 0, stream>>>(q, x.twmap, twmap_words, x.vcnt, x.vidx);
   return cudaGetLastError();
 }
 

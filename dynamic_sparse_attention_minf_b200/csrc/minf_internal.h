@@ -14,7 +14,7 @@ namespace minf {
 
 struct DevStatus;
 
-enum { POL_DENSE = 0, POL_ASHAPE = 1, POL_VS = 2, POL_BS = 3 };
+enum { POL_DENSE = 0, POL_ASHAPE = 1, POL_VS = 2, POL_BS = 3, POL_VS_EXACT = 4 };
 
 struct AttnParams {
   const __nv_bfloat16* Q;
@@ -35,6 +35,10 @@ struct AttnParams {
   const int32_t* vcnt;
   const int32_t* vidx;
   int k_s, k_v, wmap_words;
+  // element-exact Vertical-Slash (vcnt / vidx then hold per-128-row-tile lists)
+  const uint32_t* sbits;
+  const uint32_t* vbits;
+  int bits_words;
   // Block-Sparse index
   const int32_t* blk_idx;
   const int32_t* blk_cnt;
@@ -111,5 +115,7 @@ struct VsIndexParams {
   DevStatus* status;
 };
 cudaError_t vs_index_launch(const VsIndexParams& p, cudaStream_t stream);
+cudaError_t vs_exact_index_launch(const VsIndexParams& p, const minf_vs_exact_index& x, int bits_words,
+                                  int twmap_words, cudaStream_t stream);
 
 }  // namespace minf

@@ -19,11 +19,12 @@ OK = 0
 STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error",
                 4: "workspace too small", 5: "device timeout", 6: "device bounds"}
 OP_ESTIMATE_VS, OP_ESTIMATE_BS, OP_BUILD_INDEX, OP_SPARSE_ATTN_VS, OP_SPARSE_ATTN_BS, \
-    OP_ATTN_ASHAPE, OP_DENSE_ATTN = range(7)
+    OP_ATTN_ASHAPE, OP_DENSE_ATTN, OP_BUILD_INDEX_EXACT, OP_SPARSE_ATTN_VS_EXACT = range(9)
 
 EXPORTS = ["minf_vs_wmap_words", "minf_workspace_size", "minf_estimate_vs", "minf_estimate_bs",
            "minf_build_index", "minf_sparse_attn_vs", "minf_sparse_attn_bs", "minf_attn_ashape",
-           "minf_dense_attn", "minf_get_device_status", "minf_status_string"]
+           "minf_dense_attn", "minf_get_device_status", "minf_status_string", "minf_vs_bits_words",
+           "minf_vs_twmap_words", "minf_build_index_exact", "minf_sparse_attn_vs_exact"]
 
 
 class MinfError(RuntimeError):
@@ -42,6 +43,11 @@ class _VsIndexC(ctypes.Structure):
                 ("grp", "grp_cnt", "tgrp", "tgrp_cnt", "wmap", "vcnt", "vidx")]
 
 
+class _VsExactIndexC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("tgrp", "tgrp_cnt", "sbits", "vbits", "twmap", "vcnt", "vidx")]
+
+
 _lib = None
 
 
@@ -57,6 +63,13 @@ def lib():
         sp = ctypes.POINTER(Shape)
         L.minf_vs_wmap_words.argtypes = [i]
         L.minf_vs_wmap_words.restype = sz
+        L.minf_vs_bits_words.argtypes = [i]
+        L.minf_vs_bits_words.restype = sz
+        L.minf_vs_twmap_words.argtypes = [i]
+        L.minf_vs_twmap_words.restype = sz
+        L.minf_build_index_exact.argtypes = [sp, i, vp, i, vp, i, ctypes.POINTER(_VsExactIndexC), vp, sz, vp]
+        L.minf_sparse_attn_vs_exact.argtypes = [sp, vp, vp, vp, vp, i, ctypes.POINTER(_VsExactIndexC), i, i,
+                                                vp, vp, vp, sz, vp]
         L.minf_workspace_size.argtypes = [i, sp, i, i, i, i]
         L.minf_workspace_size.restype = sz
         L.minf_estimate_vs.argtypes = [sp, vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp]
@@ -71,7 +84,8 @@ def lib():
         L.minf_status_string.argtypes = [st]
         L.minf_status_string.restype = ctypes.c_char_p
         for fn in ("minf_estimate_vs", "minf_estimate_bs", "minf_build_index", "minf_sparse_attn_vs",
-                   "minf_sparse_attn_bs", "minf_attn_ashape", "minf_dense_attn", "minf_get_device_status"):
+                   "minf_sparse_attn_bs", "minf_attn_ashape", "minf_dense_attn", "minf_get_device_status",
+                   "minf_build_index_exact", "minf_sparse_attn_vs_exact"):
             getattr(L, fn).restype = st
         _lib = L
     return _lib
@@ -190,6 +204,50 @@ def minf_build_index(shape: Shape, v_idx, s_idx, index: VSIndex | None = None, w
     return index
 
 
+@dataclass
+class VSExactIndex:
+    """Device buffers of the element-exact Vertical-Slash index (see
+    minf_vs_exact_index): per 128-row query tile, offset groups of gap 128,
+    offset and key bitmaps, and the verticals outside the groups' ranges."""
+    tgrp: torch.Tensor
+    tgrp_cnt: torch.Tensor
+    sbits: torch.Tensor
+    vbits: torch.Tensor
+    twmap: torch.Tensor
+    vcnt: torch.Tensor
+    vidx: torch.Tensor
+    k_v: int
+    k_s: int
+
+    @staticmethod
+    def empty(B, nh, N, k_v, k_s, device="cuda"):
+        i32 = dict(dtype=torch.int32, device=device)
+        Wb, Wt = lib().minf_vs_bits_words(N), lib().minf_vs_twmap_words(N)
+        return VSExactIndex(torch.empty(B, nh, k_s, 2, **i32), torch.empty(B, nh, **i32),
+                            torch.empty(B, nh, Wb, **i32), torch.empty(B, nh, Wb, **i32),
+                            torch.empty(B, nh, Wt, **i32), torch.empty(B, nh, N // 128, **i32),
+                            torch.empty(B, nh, N // 128, k_v, **i32), k_v, k_s)
+
+    def c(self):
+        return _VsExactIndexC(*(t.data_ptr() for t in (self.tgrp, self.tgrp_cnt, self.sbits, self.vbits,
+                                                       self.twmap, self.vcnt, self.vidx)))
+
+
+def minf_build_index_exact(shape: Shape, v_idx, s_idx, index: VSExactIndex | None = None, ws=None,
+                           stream=None):
+    B, nh, k_v = v_idx.shape
+    k_s = s_idx.shape[2]
+    if index is None:
+        index = VSExactIndex.empty(B, nh, shape.N, k_v, k_s, device=v_idx.device)
+    if ws is None:
+        ws = workspace(OP_BUILD_INDEX_EXACT, shape, nh, device=v_idx.device)
+    ic = index.c()
+    _check("minf_build_index_exact", lib().minf_build_index_exact(
+        ctypes.byref(shape), nh, _p(v_idx), k_v, _p(s_idx), k_s, ctypes.byref(ic), _p(ws), ws.numel(),
+        _stream(stream)))
+    return index
+
+
 def _out(q, o, lse, want_lse):
     if o is None:
         o = torch.empty_like(q)
@@ -208,6 +266,21 @@ def minf_sparse_attn_vs(q, k, v, heads, index: VSIndex, o=None, lse=None, want_l
         ws = workspace(OP_SPARSE_ATTN_VS, shp, nh, device=q.device)
     ic = index.c()
     _check("minf_sparse_attn_vs", lib().minf_sparse_attn_vs(
+        ctypes.byref(shp), _p(q), _p(k), _p(v), _p(hd), nh, ctypes.byref(ic), index.k_v, index.k_s,
+        _p(o), _p(lse), _p(ws), ws.numel(), _stream(stream)))
+    return o, lse
+
+
+def minf_sparse_attn_vs_exact(q, k, v, heads, index: VSExactIndex, o=None, lse=None, want_lse=True,
+                              scale=0.0, ws=None, stream=None):
+    shp = shape_of(q, k, scale)
+    hd = _heads(heads, q.device)
+    nh = hd.numel()
+    o, lse = _out(q, o, lse, want_lse)
+    if ws is None:
+        ws = workspace(OP_SPARSE_ATTN_VS_EXACT, shp, nh, device=q.device)
+    ic = index.c()
+    _check("minf_sparse_attn_vs_exact", lib().minf_sparse_attn_vs_exact(
         ctypes.byref(shp), _p(q), _p(k), _p(v), _p(hd), nh, ctypes.byref(ic), index.k_v, index.k_s,
         _p(o), _p(lse), _p(ws), ws.numel(), _stream(stream)))
     return o, lse

@@ -227,6 +227,67 @@ minf_status minf_dense_attn(const minf_shape* shape, const minf_bf16* Q, const m
                             const minf_bf16* V, const int32_t* heads, int nh, minf_bf16* O,
                             float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Element-exact Vertical-Slash variant.  The slash lines of the summary page
+ * ("Key points": vertical and slash lines), read as the diagonals themselves
+ * rather than as the 64-key bands they sweep through a 64-row query block:
+ * row i attends to the keys j <= i with j in V or i - j in S.  This set is
+ * contained in the band set of minf_sparse_attn_vs.
+ * ------------------------------------------------------------------------- */
+enum { MINF_OP_BUILD_INDEX_EXACT = 7, MINF_OP_SPARSE_ATTN_VS_EXACT = 8 };
+
+/*
+ * Index of the exact variant, written by minf_build_index_exact and read by
+ * minf_sparse_attn_vs_exact.  Caller-owned device buffers; nt = N / 128,
+ * Wb = minf_vs_bits_words(N), Wt = minf_vs_twmap_words(N):
+ *   tgrp     [B, nh, k_s, 2] offsets merged while they differ by <= 128; the
+ *                            diagonals of group g cross the 128-row query tile
+ *                            with first row R in the keys [R - b_g, R + 127 - a_g]
+ *   tgrp_cnt [B, nh]
+ *   sbits    [B, nh, Wb]     bit o set iff offset o is in S (padding bits zero)
+ *   vbits    [B, nh, Wb]     bit j set iff key j is in V (padding bits zero)
+ *   twmap    [B, nh, Wt]     bit x set iff x lies in some [a_g, b_g + 127]; key j
+ *                            lies in one of the ranges of tile R exactly when
+ *                            bit (R + 127 - j) is set
+ *   vcnt     [B, nh, nt]     per 128-row query tile, the number of vertical
+ *                            columns outside every range of that tile
+ *   vidx     [B, nh, nt, k_v] those columns, ascending (j <= R + 127)
+ */
+typedef struct {
+  int32_t* tgrp;
+  int32_t* tgrp_cnt;
+  uint32_t* sbits;
+  uint32_t* vbits;
+  uint32_t* twmap;
+  int32_t* vcnt;
+  int32_t* vidx;
+} minf_vs_exact_index;
+
+/* Words of one head's sbits / vbits (N / 32 + 8) and of its twmap. */
+size_t minf_vs_bits_words(int N);
+size_t minf_vs_twmap_words(int N);
+
+/*
+ * Builds minf_vs_exact_index from ascending v_idx [B, nh, k_v] and s_idx
+ * [B, nh, k_s] (as minf_estimate_vs writes them).  Unsorted or out-of-range
+ * input indices set MINF_ERR_DEVICE_BOUNDS.  N must be a multiple of 128.
+ */
+minf_status minf_build_index_exact(const minf_shape* shape, int nh, const int32_t* v_idx, int k_v,
+                                   const int32_t* s_idx, int k_s, const minf_vs_exact_index* idx,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Element-exact Vertical-Slash sparse attention: row i attends to the keys
+ * j <= i with j in V or i - j in S (see above).  The key tiles are those of
+ * minf_sparse_attn_vs at 128-row granularity (the ranges of the offset groups,
+ * then the tile's vertical list); inside a range the membership of each
+ * element is read from sbits and vbits.  lse may be NULL.
+ */
+minf_status minf_sparse_attn_vs_exact(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K,
+                                      const minf_bf16* V, const int32_t* heads, int nh,
+                                      const minf_vs_exact_index* idx, int k_v, int k_s, minf_bf16* O,
+                                      float* lse, void* ws, size_t ws_bytes, void* stream);
+
 /*
  * Synchronizes `stream`, returns the device status word of `ws` (MINF_OK when
  * no kernel reported an error since the last call) and clears it.

@@ -243,3 +243,89 @@ def test_vs_estimation_long_rows(N, k_v, k_s):
         assert np.all(np.diff(gv[h]) > 0) and np.all(np.diff(gs[h]) > 0)
         check_index_set(gv[h], ov, rv, what=f"vertical h{h}")
         check_index_set(gs[h], os_, rs, forced=0, what=f"slash h{h}")
+
+
+# ------------------------------------------- element-exact Vertical-Slash
+def _vs_exact_check(w, heads, V_sets, S_sets, q, k, v, qn, kn, vn):
+    """Build the exact index from per-head (V, S), check it bit-exactly against
+    the oracle's, run the exact attention and compare with mask_vs_exact."""
+    k_v = max(len(x) for x in V_sets)
+    k_s = max(len(x) for x in S_sets)
+    assert all(len(x) == k_v for x in V_sets) and all(len(x) == k_s for x in S_sets)
+    v_idx = torch.tensor(np.stack(V_sets)[None], dtype=torch.int32, device=DEV)
+    s_idx = torch.tensor(np.stack(S_sets)[None], dtype=torch.int32, device=DEV)
+    shp = minf.shape_of(q, k)
+    ws_i = minf.workspace(minf.OP_BUILD_INDEX_EXACT, shp, len(heads))
+    index = minf.minf_build_index_exact(shp, v_idx, s_idx, ws=ws_i)
+    assert minf.minf_get_device_status(ws_i) == 0
+    nt = w.N // 128
+    for hi in range(len(heads)):
+        V, S = np.asarray(V_sets[hi]), np.asarray(S_sets[hi])
+        groups, vcnt, vidx = orc.vs_exact_index(V, S, w.N)
+        T = int(index.tgrp_cnt[0, hi])
+        assert T == groups.shape[0] and np.array_equal(index.tgrp[0, hi, :T].cpu().numpy(), groups)
+        assert np.array_equal(index.vcnt[0, hi].cpu().numpy(), vcnt)
+        gvi = index.vidx[0, hi].cpu().numpy()
+        for t in range(nt):
+            assert np.array_equal(gvi[t, :vcnt[t]], vidx[t, :vcnt[t]]), f"tile {t}"
+        sb = index.sbits[0, hi].cpu().numpy().view(np.uint32)
+        vb = index.vbits[0, hi].cpu().numpy().view(np.uint32)
+        bits = lambda words, n: np.unpackbits(words.view(np.uint8), bitorder="little")[:n].astype(bool)
+        ref_s = np.zeros(w.N, bool); ref_s[S] = True
+        ref_v = np.zeros(w.N, bool); ref_v[V] = True
+        assert np.array_equal(bits(sb, w.N), ref_s) and not bits(sb, 32 * sb.size)[w.N:].any()
+        assert np.array_equal(bits(vb, w.N), ref_v) and not bits(vb, 32 * vb.size)[w.N:].any()
+    ws_a = minf.workspace(minf.OP_SPARSE_ATTN_VS_EXACT, shp, len(heads))
+    o, lse = minf.minf_sparse_attn_vs_exact(q, k, v, heads, index, ws=ws_a)
+    assert minf.minf_get_device_status(ws_a) == 0
+    _check_attn(o, lse, qn, kn, vn, heads, w,
+                lambda hi, h: (lambda r: orc.mask_vs_exact(r, w.N, V_sets[hi], S_sets[hi])))
+    return o, lse
+
+
+def test_vs_exact_pipeline_small():
+    """Estimated V and S (GPU top-k, checked against the oracle), then the exact variant."""
+    w = wl.small(Hq=4, Hkv=2, N=2048, d=128, seed=41, k_v=64, k_s=128)
+    q, k, v, qn, kn, vn = _inputs(w)
+    sc = orc.default_scale(w.d)
+    heads = [1, 2]
+    v_idx, s_idx = minf.minf_estimate_vs(q, k, heads, w.k_v, w.k_s)
+    gv, gs = v_idx[0].cpu().numpy(), s_idx[0].cpu().numpy()
+    for hi, h in enumerate(heads):
+        rv, rs = orc.vs_estimate(qn[h][w.N - 64:], kn[orc.kv_head(h, w.Hq, w.Hkv)], sc)
+        ov, os_ = orc.vs_select(rv, rs, w.k_v, w.k_s)
+        check_index_set(gv[hi], ov, rv, what=f"vertical h{h}")
+        check_index_set(gs[hi], os_, rs, forced=0, what=f"slash h{h}")
+    _vs_exact_check(w, heads, list(gv), list(gs), q, k, v, qn, kn, vn)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_vs_exact_oracle_sets(d):
+    """Oracle-chosen sets: a long run of small offsets, scattered offsets with
+    wide gaps, and verticals inside and outside the offset ranges."""
+    w = wl.small(Hq=2, Hkv=1, N=4096, d=d, seed=42 + d)
+    q, k, v, qn, kn, vn = _inputs(w)
+    rng = np.random.default_rng(d)
+    S = np.unique(np.concatenate([[0], np.arange(1, 300), rng.choice(4096, 300, replace=False)]))[:500]
+    V = np.unique(rng.choice(4096, 200, replace=False))[:180]
+    S2 = np.unique(np.concatenate([[0], rng.choice(4096, 600, replace=False)]))[:500]
+    V2 = np.unique(np.concatenate([np.arange(0, 64), rng.choice(4096, 200, replace=False)]))[:180]
+    _vs_exact_check(w, [0, 1], [V, V2], [S, S2], q, k, v, qn, kn, vn)
+
+
+def test_vs_exact_all_offsets_equals_dense():
+    w = wl.small(Hq=2, Hkv=1, N=512, d=64, seed=43)
+    q, k, v, qn, kn, vn = _inputs(w)
+    V = np.arange(8)
+    S = np.arange(512)
+    o, lse = _vs_exact_check(w, [0, 1], [V, V], [S, S], q, k, v, qn, kn, vn)
+    od, ld = minf.minf_dense_attn(q, k, v)
+    assert (o.float() - od.float()).abs().max().item() <= 1e-2
+    assert (lse - ld).abs().max().item() <= 1e-3
+
+
+def test_vs_exact_minimum_size():
+    w = wl.small(Hq=2, Hkv=1, N=128, d=128, seed=44)
+    q, k, v, qn, kn, vn = _inputs(w)
+    _vs_exact_check(w, [0, 1], [np.array([3, 77]), np.array([0, 127])],
+                    [np.array([0, 5, 64]), np.array([0, 1, 2])], q, k, v, qn, kn, vn)
