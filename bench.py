@@ -327,21 +327,17 @@ def run_ours(args, dist, rank, world, local):
     hq.copy_(q)
     hk.copy_(k)
     hv.copy_(v)
-    e2e_steps = max(1, min(args.steps, 3))
+    e2e_steps = max(3, min(args.steps, 5))
+    pbufs = layer.PipelineBuffers(hq, hk, hv, ho, dev)
+    layer.run_pipelined(plan, hq, hk, hv, ho, 2, pbufs, compute=stream)   # warm the copy streams
     _barrier(dist)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        layer.run_layer(plan, q, k, v, o)
-        ho.copy_(o, non_blocking=True)
-    e1.record(stream)
+    e1 = layer.run_pipelined(plan, hq, hk, hv, ho, e2e_steps, pbufs, compute=stream, start_event=e0)
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(dist, e0.elapsed_time(e1) / e2e_steps)
+    del pbufs
     h2d = (q.numel() + k.numel() + v.numel()) * 2
     d2h = o.numel() * 2
 
@@ -431,7 +427,10 @@ def run_ours(args, dist, rank, world, local):
                      "peak_source": f"{src} bf16_tflops_sustained", "ms_per_launch": vs_ms,
                      "executed_tflop_per_launch": vs_exec / 1e12},
         "e2e": {"value": _throughput(world, useful, e2e_ms), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "steps": e2e_steps,
+                "mode": "layer.run_pipelined: every step uploads its Q/K/V from pinned host memory and "
+                        "downloads its O, on copy streams overlapping the neighbouring steps' compute"},
         "gpu_launches": layer.launches_per_step(plan) * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,

@@ -132,6 +132,55 @@ def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None, marks=None):
     return o, lse
 
 
+class PipelineBuffers:
+    """Two device copies of a layer's Q, K, V and O for :func:`run_pipelined`."""
+
+    def __init__(self, hq, hk, hv, ho, device):
+        self.sets = [tuple(torch.empty(x.shape, dtype=x.dtype, device=device) for x in (hq, hk, hv, ho))
+                     for _ in range(2)]
+
+
+def run_pipelined(plan: LayerPlan, hq, hk, hv, ho, steps: int, bufs: PipelineBuffers,
+                  compute=None, start_event=None):
+    """Runs the layer ``steps`` times on host-resident (pinned) inputs, end to
+    end: every step copies its Q, K and V to the device and its O back to the
+    host.  The copies run on their own streams (one per direction) into two
+    alternating device buffer sets, so that step s+1's inputs upload and step
+    s-1's output downloads while step s computes.  Work is queued behind
+    ``start_event`` (if given) on the ``compute`` stream; returns the event
+    recorded there once the last output has reached the host."""
+    compute = compute or torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    if start_event is not None:
+        up.wait_event(start_event)
+        compute.wait_event(start_event)
+    ev_in = [torch.cuda.Event() for _ in range(steps)]
+    ev_done = [torch.cuda.Event() for _ in range(steps)]
+    ev_out = [torch.cuda.Event() for _ in range(steps)]
+    for s_ in range(steps):
+        q, k, v, o = bufs.sets[s_ % 2]
+        with torch.cuda.stream(up):
+            if s_ >= 2:
+                up.wait_event(ev_done[s_ - 2])      # step s-2 has read these inputs
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            ev_in[s_].record(up)
+        compute.wait_event(ev_in[s_])
+        if s_ >= 2:
+            compute.wait_event(ev_out[s_ - 2])      # step s-2's output is on the host
+        run_layer(plan, q, k, v, o, stream=compute)
+        ev_done[s_].record(compute)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_done[s_])
+            ho.copy_(o, non_blocking=True)
+            ev_out[s_].record(down)
+    compute.wait_event(ev_out[steps - 1])
+    end = torch.cuda.Event(enable_timing=True)
+    end.record(compute)
+    return end
+
+
 def device_status(plan: LayerPlan):
     """First device-side error code across the plan's workspaces (0 = none)."""
     for name, t in plan.bufs.items():

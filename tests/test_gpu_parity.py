@@ -329,3 +329,23 @@ def test_vs_exact_minimum_size():
     q, k, v, qn, kn, vn = _inputs(w)
     _vs_exact_check(w, [0, 1], [np.array([3, 77]), np.array([0, 127])],
                     [np.array([0, 5, 64]), np.array([0, 1, 2])], q, k, v, qn, kn, vn)
+
+
+def test_pipelined_layer_matches_direct_run():
+    """layer.run_pipelined (host inputs, two device buffer sets, copy streams)
+    produces the same output as run_layer on device inputs."""
+    from dynamic_sparse_attention_minf_b200 import layer
+    w = wl.small(Hq=4, Hkv=2, N=1024, d=128, seed=51, k_v=64, k_s=96, k_b=4, n_sink=16, n_local=128,
+                 patterns=[wl.PAT_VS, wl.PAT_BS, wl.PAT_A, wl.PAT_VS])
+    q, k, v = wl.make_qkv(w, DEV)
+    plan = layer.make_plan(w, DEV)
+    o_ref = torch.empty_like(q)
+    layer.run_layer(plan, q, k, v, o_ref)
+    torch.cuda.synchronize()
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    ho = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    bufs = layer.PipelineBuffers(hq, hk, hv, ho, DEV)
+    layer.run_pipelined(plan, hq, hk, hv, ho, 3, bufs)
+    torch.cuda.synchronize()
+    assert layer.device_status(plan) == 0
+    assert torch.equal(ho, o_ref.cpu())
