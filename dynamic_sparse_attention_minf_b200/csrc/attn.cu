@@ -760,18 +760,22 @@ __global__ void __launch_bounds__(320, 1)
         if (!mbar_wait(&p_full[bp], (tp >> 1) & 1, abort, p.status, 3)) return false;
         if (!mbar_wait(&v_full[sp], (tp / C::kStages) & 1, abort, p.status, 4)) return false;
         tc_fence_after();
-        const uint32_t vaddr = smem_u32(smem + C::kOffV + sp * C::kKVBytes);
+        // descriptors of the K-steps: the stage's base plus a constant (the
+        // start-address field holds address / 16 and never carries out)
+        const uint64_t vd0 = sdesc_sw128(smem_u32(smem + C::kOffV + sp * C::kKVBytes), C::kRegion, 1024);
+        const uint32_t a0 = tmem + bp * 128;
+        const uint32_t acc0 = tp > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, C::kRegion, 1024);
           const uint32_t d_tmem = tmem + (kk < 4 ? C::kColO0 : C::kColO1);
-          const uint32_t a_tmem = tmem + bp * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
-          umma_ts(d_tmem, a_tmem, bd, C::kIdescPV, (tp > 0 || (kk & 3) > 0) ? 1u : 0u);
+          umma_ts(d_tmem, a0 + (kk >> 2) * 64 + (kk & 3) * 8, vd0 + (uint64_t)(kk * 2048 / 16), C::kIdescPV,
+                  (kk & 3) > 0 ? 1u : acc0);
         }
         umma_commit(&v_empty[sp]);
         return true;
       };
       bool ok = mbar_wait(q_full, 0, abort, p.status, 2);
+      const uint64_t qd0 = sdesc_sw128(qaddr, 16, 1024);
       int t = 0, pend = -1;
       while (ok) {
         const int st = t % C::kStages;
@@ -781,13 +785,11 @@ __global__ void __launch_bounds__(320, 1)
         // fence; the barrier alone orders them before the MMA (no tcgen05
         // fence here: it would stall the issue of every tile).
         const int w = t & 1;  // S buffer
-        const uint32_t kaddr = smem_u32(smem + C::kOffK + st * C::kKVBytes);
+        const uint64_t kd0 = sdesc_sw128(smem_u32(smem + C::kOffK + st * C::kKVBytes), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kRegion + (kk & 3) * 32;
-          const uint64_t ad = sdesc_sw128(qaddr + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(kaddr + off, 16, 1024);
-          umma_ss(tmem + w * 128, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
+          const uint64_t off16 = (uint64_t)(((kk >> 2) * C::kRegion + (kk & 3) * 32) / 16);
+          umma_ss(tmem + w * 128, qd0 + off16, kd0 + off16, C::kIdescS, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[w]);
         umma_commit(&k_empty[st]);
