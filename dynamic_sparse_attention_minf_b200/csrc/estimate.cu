@@ -292,7 +292,36 @@ __device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long 
   return v + before;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_rows_kernel(const TopkRows t) {
+// The digit of the rem-th largest key from an NB-bin histogram (all threads
+// of the block take part): returns the digit and the count of keys in higher
+// digits (through shared memory).
+__device__ void topk_find_digit(const unsigned* h, int NB, uint32_t rem, unsigned long long* wsum,
+                                uint32_t* sh_digit, uint32_t* sh_above) {
+  const int per = NB / blockDim.x;  // bins per thread, descending
+  uint32_t sum = 0;
+  for (int e = 0; e < per; ++e) sum += h[NB - 1 - per * threadIdx.x - e];
+  unsigned long long tot;
+  const unsigned long long inc = block_scan_u64(sum, wsum, tot);
+  const unsigned long long before = inc - sum;
+  if (before < rem && inc >= rem) {
+    uint32_t cum = (uint32_t)before;
+    for (int e = 0; e < per; ++e) {
+      const uint32_t c = h[NB - 1 - per * threadIdx.x - e];
+      if (cum + c >= rem) {
+        *sh_digit = (uint32_t)(NB - 1 - per * threadIdx.x - e);
+        *sh_above = cum;
+        break;
+      }
+      cum += c;
+    }
+  }
+  __syncthreads();
+}
+
+constexpr int kTopkCap = 1024;  // candidate buffer of the short-row path
+
+template <bool SHORT>
+__device__ __forceinline__ void topk_rows_body(const TopkRows& t) {
   const int row = blockIdx.x;
   const int len = (t.len_mode == 0) ? t.len : (row % t.rows_per_group) + 1;
   const int forced = (t.forced_mode == 0) ? -1 : (t.forced_mode == 1) ? 0 : (row % t.rows_per_group);
@@ -301,7 +330,113 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_rows_kernel(const TopkRo
   __shared__ unsigned hist[kTopkThreads / 32][256];  // one histogram per warp
   __shared__ unsigned long long wsum[32];
   __shared__ uint32_t sh_sel, sh_rem;
+  __shared__ uint32_t ck[kTopkCap];
+  __shared__ int32_t ci[kTopkCap];
   auto key_of = [&](int j) -> uint32_t { return (j == forced) ? 0xFFFFFFFFu : order_key(sc[j]); };
+
+  // Short rows: two passes over the row.  (1) a histogram of the top 11 key
+  // bits gives the bin of the k-th largest key; (2) every key in that bin or
+  // above (fewer than k above, plus the bin) is copied in index order to
+  // shared memory.  The threshold is then resolved within those candidates
+  // and they are compacted in order.  Rows whose candidates do not fit take
+  // the general path below.
+  if (SHORT && k > 0) {
+    unsigned* h = &hist[0][0];  // 2048 bins
+    for (int x = threadIdx.x; x < 2048; x += blockDim.x) h[x] = 0;
+    __syncthreads();
+    {
+      uint32_t last = 2048;
+      unsigned run = 0;
+      for (int base = 0; base < len; base += blockDim.x * kTopkLoads) {
+        uint32_t dg[kTopkLoads];
+#pragma unroll
+        for (int e = 0; e < kTopkLoads; ++e) {
+          const int j = base + e * blockDim.x + threadIdx.x;
+          dg[e] = (j < len) ? (key_of(j) >> 21) : 2048u;
+        }
+#pragma unroll
+        for (int e = 0; e < kTopkLoads; ++e) {
+          if (dg[e] != last) {
+            if (last < 2048) atomicAdd(&h[last], run);
+            last = dg[e];
+            run = 0;
+          }
+          ++run;
+        }
+      }
+      if (last < 2048) atomicAdd(&h[last], run);
+    }
+    __syncthreads();
+    topk_find_digit(h, 2048, (uint32_t)k, wsum, &sh_sel, &sh_rem);
+    const uint32_t b1 = sh_sel, above = sh_rem;
+    const uint32_t M = above + h[b1];
+    __syncthreads();
+    if (M <= (uint32_t)kTopkCap) {
+      // (2) ordered copy of the keys with top bits >= b1
+      unsigned long long taken = 0;
+      const int chunk = blockDim.x * kTopkItems;
+      for (int base = 0; base < len; base += chunk) {
+        uint32_t keys[kTopkItems];
+        unsigned c = 0;
+#pragma unroll
+        for (int e = 0; e < kTopkItems; ++e) {
+          const int j = base + threadIdx.x * kTopkItems + e;
+          keys[e] = (j < len) ? key_of(j) : 0u;
+          c += (j < len && (keys[e] >> 21) >= b1);
+        }
+        unsigned long long tot;
+        const unsigned long long inc = block_scan_u64(c, wsum, tot);
+        unsigned long long pos = taken + inc - c;
+#pragma unroll
+        for (int e = 0; e < kTopkItems; ++e) {
+          const int j = base + threadIdx.x * kTopkItems + e;
+          if (j < len && (keys[e] >> 21) >= b1) {
+            ck[pos] = keys[e];
+            ci[pos] = j;
+            ++pos;
+          }
+        }
+        taken += tot;
+      }
+      __syncthreads();
+      // the exact threshold among the bin's keys: 11 more bits, then 10
+      uint32_t prefix = b1 << 21, pmask = 0xFFE00000u, rem = (uint32_t)k - above;
+      for (int pass = 0; pass < 2; ++pass) {
+        const int shift = pass == 0 ? 10 : 0, nb = pass == 0 ? 2048 : 1024;
+        for (int x = threadIdx.x; x < nb; x += blockDim.x) h[x] = 0;
+        __syncthreads();
+        for (uint32_t x = threadIdx.x; x < M; x += blockDim.x)
+          if ((ck[x] & pmask) == prefix) atomicAdd(&h[(ck[x] >> shift) & (nb - 1)], 1u);
+        __syncthreads();
+        topk_find_digit(h, nb, rem, wsum, &sh_sel, &sh_rem);
+        prefix |= sh_sel << shift;
+        pmask |= (uint32_t)(nb - 1) << shift;
+        rem -= sh_rem;
+        __syncthreads();
+      }
+      const uint32_t T = prefix;
+      const uint32_t need = rem;  // keys equal to T that are taken (lowest indices)
+      // ordered compaction of the candidates
+      int32_t* out = t.out_idx + (long long)row * t.k;
+      unsigned long long gt_before = 0, eq_before = 0;
+      for (uint32_t base = 0; base < M; base += blockDim.x) {
+        const uint32_t x = base + threadIdx.x;
+        const uint32_t key = (x < M) ? ck[x] : 0u;
+        const unsigned cg = (x < M && key > T), ce = (x < M && key == T);
+        unsigned long long tot;
+        const unsigned long long inc = block_scan_u64(((unsigned long long)cg << 32) | ce, wsum, tot);
+        const unsigned long long exc = inc - (((unsigned long long)cg << 32) | ce);
+        const unsigned long long g = gt_before + (exc >> 32), q = eq_before + (exc & 0xFFFFFFFFull);
+        if (cg) out[g + min(q, (unsigned long long)need)] = ci[x];
+        else if (ce && q < need) out[g + q] = ci[x];
+        gt_before += tot >> 32;
+        eq_before += tot & 0xFFFFFFFFull;
+      }
+      for (int x = k + threadIdx.x; x < t.k; x += blockDim.x) out[x] = -1;
+      if (t.out_cnt && threadIdx.x == 0) t.out_cnt[row] = k;
+      return;
+    }
+  }
 
   // radix select of the k-th largest key, 8 bits at a time from the top
   uint32_t prefix = 0, pmask = 0, rem = (uint32_t)k;
@@ -425,6 +560,11 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_rows_kernel(const TopkRo
   for (int x = k + threadIdx.x; x < t.k; x += blockDim.x) out[x] = -1;
   if (t.out_cnt && threadIdx.x == 0) t.out_cnt[row] = k;
 }
+
+// One CTA per row: 1024 threads for rows too long for the short-row path
+// (only when no scratch is given), 256 for the rest.
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_rows_kernel(const TopkRows t) { topk_rows_body<false>(t); }
+__global__ void __launch_bounds__(256) topk_short_rows_kernel(const TopkRows t) { topk_rows_body<true>(t); }
 
 // ---------------------------------------------- top-k of long rows, many CTAs
 // The same selection as topk_rows_kernel, for rows too long for one CTA: the
@@ -630,8 +770,10 @@ cudaError_t topk_rows_launch(const TopkRows& t, cudaStream_t stream) {
     return topk_long_rows_launch(t, stream);
   // long rows (Vertical-Slash: one per head) take a whole SM each; short
   // rows (Block-Sparse: one per query block) run several CTAs per SM
-  const int threads = (t.len > 32768) ? kTopkThreads : 256;
-  topk_rows_kernel<<<t.rows, threads, 0, stream>>>(t);
+  if (t.len > 32768)
+    topk_rows_kernel<<<t.rows, kTopkThreads, 0, stream>>>(t);
+  else
+    topk_short_rows_kernel<<<t.rows, 256, 0, stream>>>(t);
   return cudaGetLastError();
 }
 
