@@ -114,6 +114,27 @@ def check_head(task: dict) -> dict:
                 if bad:
                     out["errors"].append(f"vidx differs in {len(bad)} blocks, e.g. {bad[:4]}")
             mask_fn = lambda r: orc.mask_vs(r, N, gv, gs)
+            if "ox_rows" in task:
+                # element-exact variant on the same sets: its per-tile vertical
+                # lists bit-exactly, its outputs on the sampled rows
+                _, xcnt, xidx = orc.vs_exact_index(gv, gs, N)
+                s_xi, XI = task["xidx"].attach(); shms.append(s_xi)
+                if not np.array_equal(task["xcnt"], xcnt):
+                    out["errors"].append("exact vcnt differs")
+                else:
+                    bad = [t for t in range(N // 128)
+                           if not np.array_equal(XI[task["slot"], t, :xcnt[t]], xidx[t, :xcnt[t]])]
+                    if bad:
+                        out["errors"].append(f"exact vidx differs in {len(bad)} tiles, e.g. {bad[:4]}")
+                q_rows = bf16_bits_to_f64(Q[h, rows])
+                OX, LX = _attention_rows(q_rows, k64, v64, rows, lambda r: orc.mask_vs_exact(r, N, gv, gs), sc)
+                ex = np.abs(task["ox_rows"].astype(np.float64) - OX)
+                out["x_max_abs"] = float(ex.max())
+                if not np.isfinite(task["ox_rows"]).all() or ex.max() > MAX_ABS or ex.mean() > MEAN_ABS:
+                    out["errors"].append(f"exact attention error max {ex.max():.3g} mean {ex.mean():.3g}")
+                lx = np.abs(task["lsex_rows"] - LX)
+                if lx[np.isfinite(LX)].max() > LSE_ABS:
+                    out["errors"].append(f"exact lse error {lx[np.isfinite(LX)].max():.3g}")
         elif pat == "bs":
             qh = bf16_bits_to_f64(Q[h])
             qbar, kbar = orc.bs_pool(qh), orc.bs_pool(k64)

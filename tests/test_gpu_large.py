@@ -1,5 +1,6 @@
 """Full-size parity: the whole mixed-pattern layer at N = 128K, 512K and 1M
-tokens, in the launch configuration bench.py times.  Index sets are checked
+tokens, in the launch configuration bench.py times, and the element-exact
+Vertical-Slash variant on the same heads and sets.  Index sets are checked
 in full (bit-exact up to the score-gap rule, the index build bit-exact);
 attention outputs on 512 seeded sampled query rows per head.  The oracle runs
 in a spawn-started process pool, one query head per task."""
@@ -38,6 +39,18 @@ def test_full_size_layer(cid):
     rows_d = rows.to("cuda")
     o_rows = o[0][:, rows_d].float().cpu().numpy()
     lse_rows = lse[0][:, rows_d].cpu().numpy()
+    # the element-exact variant on the same VS heads and sets (into the same
+    # output buffers, whose sampled rows are already copied)
+    xi = None
+    if plan.vs_heads is not None:
+        b = plan.bufs
+        ws_xi = minf.workspace(minf.OP_BUILD_INDEX_EXACT, plan.shape, plan.vs_heads.numel())
+        xi = minf.minf_build_index_exact(plan.shape, b["v_idx"], b["s_idx"], ws=ws_xi)
+        ws_x = minf.workspace(minf.OP_SPARSE_ATTN_VS_EXACT, plan.shape, plan.vs_heads.numel())
+        minf.minf_sparse_attn_vs_exact(q, k, v, plan.vs_heads, xi, o=o, lse=lse, ws=ws_x)
+        assert minf.minf_get_device_status(ws_xi) == 0 and minf.minf_get_device_status(ws_x) == 0
+        ox_rows = o[0][:, rows_d].float().cpu().numpy()
+        lsex_rows = lse[0][:, rows_d].cpu().numpy()
 
     keep = []
     try:
@@ -54,6 +67,8 @@ def test_full_size_layer(cid):
             grp, grp_cnt = idx.grp[0].cpu().numpy(), idx.grp_cnt[0].cpu().numpy()
             tgrp, tgrp_cnt = idx.tgrp[0].cpu().numpy(), idx.tgrp_cnt[0].cpu().numpy()
             vcnt = idx.vcnt[0].cpu().numpy()
+            XI = op.share(xi.vidx[0].cpu().numpy(), keep)
+            xcnt = xi.vcnt[0].cpu().numpy()
         if bs_pos:
             blk_idx, blk_cnt = b["blk_idx"][0].cpu().numpy(), b["blk_cnt"][0].cpu().numpy()
         tasks = []
@@ -63,7 +78,8 @@ def test_full_size_layer(cid):
             if h in vs_pos:
                 a = vs_pos[h]
                 t.update(pattern="vs", k_v=w.k_v, k_s=w.k_s, v_idx=v_idx[a], s_idx=s_idx[a],
-                         grp=grp[a, :grp_cnt[a]], tgrp=tgrp[a, :tgrp_cnt[a]], vcnt=vcnt[a], vidx=VI, slot=a)
+                         grp=grp[a, :grp_cnt[a]], tgrp=tgrp[a, :tgrp_cnt[a]], vcnt=vcnt[a], vidx=VI, slot=a,
+                         ox_rows=ox_rows[h], lsex_rows=lsex_rows[h], xcnt=xcnt[a], xidx=XI)
             elif h in bs_pos:
                 a = bs_pos[h]
                 t.update(pattern="bs", k_b=w.k_b, blk_idx=blk_idx[a], blk_cnt=blk_cnt[a])
