@@ -848,7 +848,10 @@ __global__ void __launch_bounds__(320, 1)
       if (exact) {
         // bit c: (i - j in S) or (j in V) for key j = j0 + c; these words
         // differ between rows, so the chunk tests below are per thread here
-        const uint64_t em = brev64(xs.bits()) | xv.bits();
+        uint64_t em = brev64(xs.bits()) | xv.bits();
+        // causal as bits: key j0 + c is allowed for c <= i - j0
+        const int lim = i - dd.j0[wg];
+        em &= (lim >= 63) ? ~0ull : (lim < 0 ? 0ull : ((2ull << lim) - 1ull));
         mw[0] &= (uint32_t)em;
         mw[1] &= (uint32_t)(em >> 32);
       }
@@ -869,7 +872,7 @@ __global__ void __launch_bounds__(320, 1)
             if (!((mw[c2] >> e) & 1u)) s[c2 * 32 + e] = -INFINITY;
         }
       }
-      if (flags & (F_CAUSAL | F_ASHAPE | F_EXACT)) {
+      if (!exact && (flags & (F_CAUSAL | F_ASHAPE))) {
         const bool causal = flags & F_CAUSAL;
         const bool ash = flags & F_ASHAPE;
         if (kind == KIND_RANGE) {
