@@ -843,11 +843,98 @@ __global__ void __launch_bounds__(256) bs_score_kernel(const BsEstParams p) {
   }
 }
 
+// t[b, c] = scale * qbar_b . kbar_c over 128 x 128 tiles of the lower
+// triangle (c-tile <= b-tile), one CTA per tile: 256 threads with 8 x 8
+// outputs each, packed two-lane fp32 FMAs, k in chunks of 16 staged
+// transposed in shared memory.
+constexpr int kBsT = 128, kBsK = 16, kBsPad = 4;
+__global__ void __launch_bounds__(256) bs_score_tri_kernel(const BsEstParams p, int nt) {
+  // lower-triangle tile x -> (bt, ct), ct <= bt
+  const int x = blockIdx.x;
+  int bt = (int)((sqrtf(8.f * (float)x + 1.f) - 1.f) * 0.5f);
+  while ((bt + 1) * (bt + 2) / 2 <= x) ++bt;
+  while (bt * (bt + 1) / 2 > x) --bt;
+  const int ct = x - bt * (bt + 1) / 2;
+  const int bhz = blockIdx.y;
+  const int nb = p.N / 64;
+  const float* qb = p.qbar + (size_t)bhz * nb * p.d;
+  const float* kb = p.kbar + (size_t)bhz * nb * p.d;
+  __shared__ __align__(16) float As[kBsK][kBsT + kBsPad];
+  __shared__ __align__(16) float Bs[kBsK][kBsT + kBsPad];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  uint64_t acc[8][4];  // row ty*8+i, columns tx*8 + 2j, 2j+1
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0ull;
+  for (int k0 = 0; k0 < p.d; k0 += kBsK) {
+    // 128 rows x 16 k of each operand: 512 float4 per operand, 2 per thread
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int f = tid + 256 * u;
+      const int r = f >> 2, kq = f & 3;
+      const int gr = bt * kBsT + r, gc = ct * kBsT + r;
+      const float4 av = (gr < nb) ? *reinterpret_cast<const float4*>(qb + (size_t)gr * p.d + k0 + 4 * kq)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 bv = (gc < nb) ? *reinterpret_cast<const float4*>(kb + (size_t)gc * p.d + k0 + 4 * kq)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      As[4 * kq + 0][r] = av.x; As[4 * kq + 1][r] = av.y; As[4 * kq + 2][r] = av.z; As[4 * kq + 3][r] = av.w;
+      Bs[4 * kq + 0][r] = bv.x; Bs[4 * kq + 1][r] = bv.y; Bs[4 * kq + 2][r] = bv.z; Bs[4 * kq + 3][r] = bv.w;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kBsK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][ty * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8 + 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const uint64_t bp[4] = {f32x2_pack(b0.x, b0.y), f32x2_pack(b0.z, b0.w), f32x2_pack(b1.x, b1.y),
+                              f32x2_pack(b1.z, b1.w)};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint64_t a2 = f32x2_pack(av[i], av[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = f32x2_fma(a2, bp[j], acc[i][j]);
+      }
+    }
+    __syncthreads();
+  }
+  float* out = p.scores + (size_t)bhz * nb * nb;
+  const int c0 = ct * kBsT + tx * 8;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = bt * kBsT + ty * 8 + i;
+    if (r >= nb) continue;
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f32x2_unpack(acc[i][j], v[2 * j], v[2 * j + 1]);
+      v[2 * j] *= p.scale;
+      v[2 * j + 1] *= p.scale;
+    }
+    if (c0 + 8 <= nb) {
+      float4* dst = reinterpret_cast<float4*>(out + (size_t)r * nb + c0);
+      dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+      dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (c0 + j < nb) out[(size_t)r * nb + c0 + j] = v[j];
+    }
+  }
+}
+
 cudaError_t bs_pool_score_launch(const BsEstParams& p, cudaStream_t stream) {
   const int nb = p.N / 64;
   bs_pool_kernel<<<dim3(nb, p.nh, p.B), 2 * p.d, 0, stream>>>(p);
-  const int nt = (nb + 63) / 64;
-  bs_score_kernel<<<dim3(nt, nt, p.B * p.nh), 256, 0, stream>>>(p);
+  if (nb % 8 == 0 && p.d % kBsK == 0) {
+    const int nt = (nb + kBsT - 1) / kBsT;
+    bs_score_tri_kernel<<<dim3(nt * (nt + 1) / 2, p.B * p.nh), 256, 0, stream>>>(p, nt);
+  } else {
+    const int nt = (nb + 63) / 64;
+    bs_score_kernel<<<dim3(nt, nt, p.B * p.nh), 256, 0, stream>>>(p);
+  }
   return cudaGetLastError();
 }
 
