@@ -14,100 +14,10 @@
 namespace minf {
 
 // ===================================================== Vertical-Slash scores
-// One CTA: 64 query rows (the last L <= 64 rows of one head) x 128 keys.
+// Row combine and slash sums of the tensor-core estimation (estimate_tc.cu):
+// score tiles of 128 keys, 192 diagonal partials per tile (191 used).
 constexpr int kVsKeys = 128;
 constexpr int kVsDiag = 192;  // diagonals of a 64 x 128 tile (191 used)
-
-template <int D>
-struct VsSmem {
-  float q[D][64];                 // transposed last rows of Q
-  float k[D][kVsKeys + 4];        // transposed key tile
-};
-
-// Scores of the CTA's 64 x 128 tile in the log2 domain: acc[a][b] holds row
-// ty*4+a, column tx*8+b.
-template <int D>
-__device__ __forceinline__ void vs_tile_scores(const VsEstParams& p, VsSmem<D>& sm, int b, int head, int kvh,
-                                               int j0, float (&acc)[4][8]) {
-  const int tid = threadIdx.x;
-  const int L = p.last_q;
-  const __nv_bfloat16* qh = p.Q + ((size_t)(b * p.Hq + head) * p.N + (p.N - L)) * D;
-  const __nv_bfloat16* kh = p.K + ((size_t)(b * p.Hkv + kvh) * p.N + j0) * D;
-  for (int e = tid; e < 64 * D; e += blockDim.x) {
-    const int r = e / D, dd = e % D;
-    sm.q[dd][r] = (r < L) ? __bfloat162float(qh[(size_t)r * D + dd]) : 0.f;
-  }
-  for (int e = tid; e < kVsKeys * D; e += blockDim.x) {
-    const int c = e / D, dd = e % D;
-    sm.k[dd][c] = (j0 + c < p.N) ? __bfloat162float(kh[(size_t)c * D + dd]) : 0.f;
-  }
-  __syncthreads();
-  const int ty = tid >> 4, tx = tid & 15;
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
-#pragma unroll 4
-  for (int dd = 0; dd < D; ++dd) {
-    const float4 qv = *reinterpret_cast<const float4*>(&sm.q[dd][ty * 4]);
-    const float4 k0 = *reinterpret_cast<const float4*>(&sm.k[dd][tx * 8]);
-    const float4 k1 = *reinterpret_cast<const float4*>(&sm.k[dd][tx * 8 + 4]);
-    const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
-    const float kb[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(qa[a], kb[c], acc[a][c]);
-  }
-  // scale into log2 units and apply the causal / range mask
-#pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int r = ty * 4 + a;
-    const int i = p.N - L + r;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int j = j0 + tx * 8 + c;
-      const bool ok = (r < L) && (j <= i) && (j < p.N);
-      acc[a][c] = ok ? acc[a][c] * p.scale_log2 : -INFINITY;
-    }
-  }
-}
-
-template <int D>
-__global__ void __launch_bounds__(256) vs_pass1_kernel(const VsEstParams p) {
-  extern __shared__ __align__(16) uint8_t smraw[];
-  VsSmem<D>& sm = *reinterpret_cast<VsSmem<D>*>(smraw);
-  const int tile = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
-  const int head = p.heads[hi];
-  if (head < 0 || head >= p.Hq) {
-    if (threadIdx.x == 0) report(p.status, MINF_ERR_DEVICE_BOUNDS, 30);
-    return;
-  }
-  float acc[4][8];
-  vs_tile_scores<D>(p, sm, b, head, head / p.group, tile * kVsKeys, acc);
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  const int ntiles = gridDim.x;
-  float* out = p.part_ml + (((size_t)(b * p.nh + hi) * ntiles + tile) * 64) * 2;
-#pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    float m = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) m = fmaxf(m, acc[a][c]);
-#pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    float l = 0.f;
-    if (m != -INFINITY) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) l += exp2f(acc[a][c] - m);
-    }
-#pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, o);
-    if (tx == 0) {
-      out[(ty * 4 + a) * 2 + 0] = m;
-      out[(ty * 4 + a) * 2 + 1] = l;
-    }
-  }
-}
 
 // Combines the per-tile (max, sum) of each row in a fixed order.
 __global__ void __launch_bounds__(256) vs_combine_kernel(const VsEstParams p, int ntiles) {
@@ -144,56 +54,6 @@ __global__ void __launch_bounds__(256) vs_combine_kernel(const VsEstParams p, in
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(256) vs_pass2_kernel(const VsEstParams p) {
-  extern __shared__ __align__(16) uint8_t smraw[];
-  VsSmem<D>& sm = *reinterpret_cast<VsSmem<D>*>(smraw);
-  const int tile = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
-  const int head = p.heads[hi];
-  if (head < 0 || head >= p.Hq) return;
-  const int j0 = tile * kVsKeys;
-  float acc[4][8];
-  vs_tile_scores<D>(p, sm, b, head, head / p.group, j0, acc);
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const float* rml = p.row_ml + (size_t)(b * p.nh + hi) * 64 * 2;
-#pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const float m = rml[(ty * 4 + a) * 2], il = rml[(ty * 4 + a) * 2 + 1];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[a][c] = (acc[a][c] == -INFINITY) ? 0.f : exp2f(acc[a][c] - m) * il;
-  }
-  __syncthreads();  // the key tile is no longer needed: reuse shared memory
-  float* P = reinterpret_cast<float*>(smraw);               // [64][129]
-  float* colp = P + 64 * 129;                               // [16][128]
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) P[(ty * 4 + a) * 129 + tx * 8 + c] = acc[a][c];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    float cs = 0.f;
-#pragma unroll
-    for (int a = 0; a < 4; ++a) cs += acc[a][c];
-    colp[ty * 128 + tx * 8 + c] = cs;
-  }
-  __syncthreads();
-  const size_t bh = (size_t)(b * p.nh + hi);
-  if (tid < kVsKeys) {
-    float v = 0.f;
-#pragma unroll
-    for (int y = 0; y < 16; ++y) v += colp[y * 128 + tid];
-    if (j0 + tid < p.N) p.v_score[bh * p.N + j0 + tid] = v;
-  }
-  // diagonal k = r - c + 127 of the tile, summed over rows in ascending order
-  if (tid < 191) {
-    const int k = tid;
-    float dsum = 0.f;
-    const int rlo = max(0, k - 127), rhi = min(63, k);
-    for (int r = rlo; r <= rhi; ++r) dsum += P[r * 129 + (r - k + 127)];
-    p.dpart[(bh * gridDim.x + tile) * kVsDiag + k] = dsum;
-  }
-}
-
 // sigma_o = sum of the (at most two) tiles' diagonal partials holding offset o.
 __global__ void __launch_bounds__(256) vs_slash_kernel(const VsEstParams p, int ntiles) {
   const int o = blockIdx.x * 256 + threadIdx.x;
@@ -221,35 +81,6 @@ cudaError_t vs_combine_launch(const VsEstParams& p, int nparts, cudaStream_t str
 
 cudaError_t vs_slash_launch(const VsEstParams& p, cudaStream_t stream) {
   const int ntiles = (p.N + kVsKeys - 1) / kVsKeys;
-  vs_slash_kernel<<<dim3((p.N + 255) / 256, p.nh, p.B), 256, 0, stream>>>(p, ntiles);
-  return cudaGetLastError();
-}
-
-cudaError_t vs_estimate_launch(const VsEstParams& p, cudaStream_t stream) {
-  const int ntiles = (p.N + kVsKeys - 1) / kVsKeys;
-  dim3 grid(ntiles, p.nh, p.B);
-  size_t sm = (p.d == 128) ? sizeof(VsSmem<128>) : sizeof(VsSmem<64>);
-  const size_t sm2 = (64 * 129 + 16 * 128) * sizeof(float);
-  if (sm < sm2) sm = sm2;
-  cudaError_t e;
-  if (p.d == 128) {
-    e = cudaFuncSetAttribute(vs_pass1_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(vs_pass2_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    vs_pass1_kernel<128><<<grid, 256, sm, stream>>>(p);
-  } else {
-    e = cudaFuncSetAttribute(vs_pass1_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(vs_pass2_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    vs_pass1_kernel<64><<<grid, 256, sm, stream>>>(p);
-  }
-  vs_combine_kernel<<<dim3(64, p.nh, p.B), 256, 0, stream>>>(p, ntiles);
-  if (p.d == 128)
-    vs_pass2_kernel<128><<<grid, 256, sm, stream>>>(p);
-  else
-    vs_pass2_kernel<64><<<grid, 256, sm, stream>>>(p);
   vs_slash_kernel<<<dim3((p.N + 255) / 256, p.nh, p.B), 256, 0, stream>>>(p, ntiles);
   return cudaGetLastError();
 }

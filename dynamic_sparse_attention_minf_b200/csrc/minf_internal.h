@@ -65,7 +65,6 @@ struct VsEstParams {
   float* s_score;     // [B, nh, N]
   DevStatus* status;
 };
-cudaError_t vs_estimate_launch(const VsEstParams& p, cudaStream_t stream);
 cudaError_t vs_combine_launch(const VsEstParams& p, int nparts, cudaStream_t stream);
 cudaError_t vs_slash_launch(const VsEstParams& p, cudaStream_t stream);
 // tensor-core estimation: tq and tk view Q and K as [rows, d] with 64-row
