@@ -6,9 +6,12 @@
 //   warp  8    tcgen05 issuer (one lane) and TMEM owner
 //   warp  9    producer: enumerates the key tiles of the query tile for the
 //              head's pattern, writes each tile's descriptor (column ids and
-//              per-64-row-half membership masks) and stages K/V into shared
-//              memory by TMA (contiguous 64-key chunks) or cp.async (gathered
-//              columns).
+//              per-64-row-half membership masks) and stages K and V into two
+//              rings of shared-memory slots: by TMA for contiguous 64-key
+//              chunks (one 128-row box when the two chunks are adjacent), by
+//              cp.async for gathered columns.  A K slot frees when S of its
+//              tile is done, a V slot when P V is; the V of a range tile is
+//              loaded after the next tile's K.
 //
 // Per key tile t (128 keys) the issuer computes S = Q K^T into TMEM buffer
 // t&1.  Warpgroup w masks and exponentiates its 64 columns of S and writes P
@@ -27,6 +30,13 @@
 //   VS      : the union over slash groups of the bands swept by the tile's
 //             rows, then the verticals of both 64-row halves, gathered
 //   BS      : the selected 64-key blocks of both halves, two per tile
+//   VS exact: the same ranges at 128-row granularity, masked per element
+//             from offset and key bitmaps, then the tile's vertical list
+//
+// The softmax runs one pair of exponentials in four through a polynomial on
+// the FMA pipe (the rest on the MUFU).  Every wait is bounded: a wait that
+// runs out records MINF_ERR_DEVICE_TIMEOUT, and all roles stop, drain their
+// copies and MMAs, free TMEM and return.
 #include "minf_device.cuh"
 #include "minf_internal.h"
 
