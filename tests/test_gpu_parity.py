@@ -349,3 +349,50 @@ def test_pipelined_layer_matches_direct_run():
     torch.cuda.synchronize()
     assert layer.device_status(plan) == 0
     assert torch.equal(ho, o_ref.cpu())
+
+
+# ------------------------------------------------------------- batch > 1
+def test_batch_of_two_every_entry_point():
+    """B = 2: every entry point, each batch element against the oracle on its
+    own inputs (the kernels index the batch by grid z)."""
+    w = wl.small(Hq=4, Hkv=2, N=1024, d=128, seed=61, k_v=48, k_s=96, k_b=4, B=2)
+    q, k, v = wl.make_qkv(w, DEV)
+    assert q.shape[0] == 2
+    sc = orc.default_scale(w.d)
+    shp = minf.shape_of(q, k)
+    heads = [1, 2]
+    # Vertical-Slash: estimation, index, attention (band and exact)
+    v_idx, s_idx, vsc, ssc = minf.minf_estimate_vs(q, k, heads, w.k_v, w.k_s, return_scores=True)
+    index = minf.minf_build_index(shp, v_idx, s_idx)
+    o_vs, l_vs = minf.minf_sparse_attn_vs(q, k, v, heads, index)
+    xi = minf.minf_build_index_exact(shp, v_idx, s_idx)
+    o_x, l_x = minf.minf_sparse_attn_vs_exact(q, k, v, heads, xi)
+    # Block-Sparse, A-shape, dense
+    blk_idx, blk_cnt = minf.minf_estimate_bs(q, k, heads, w.k_b)
+    o_bs, l_bs = minf.minf_sparse_attn_bs(q, k, v, heads, blk_idx, blk_cnt)
+    o_a, l_a = minf.minf_attn_ashape(q, k, v, heads, 16, 100)
+    o_d, l_d = minf.minf_dense_attn(q, k, v)
+    torch.cuda.synchronize()
+    rows = np.arange(w.N)
+    for bb in range(2):
+        qn, kn, vn = orc.to_f64(q[bb]), orc.to_f64(k[bb]), orc.to_f64(v[bb])
+        gv, gs = v_idx[bb].cpu().numpy(), s_idx[bb].cpu().numpy()
+        gi, gc = blk_idx[bb].cpu().numpy(), blk_cnt[bb].cpu().numpy()
+        for hi, h in enumerate(heads):
+            kv = orc.kv_head(h, w.Hq, w.Hkv)
+            rv, rs = orc.vs_estimate(qn[h][w.N - 64:], kn[kv], sc)
+            np.testing.assert_allclose(vsc[bb, hi].cpu().numpy(), rv, rtol=1e-4, atol=1e-7)
+            ov, os_ = orc.vs_select(rv, rs, w.k_v, w.k_s)
+            check_index_set(gv[hi], ov, rv, what=f"b{bb} vertical h{h}")
+            check_index_set(gs[hi], os_, rs, forced=0, what=f"b{bb} slash h{h}")
+            cases = [
+                (o_vs, l_vs, lambda r: orc.mask_vs(r, w.N, gv[hi], gs[hi]), "vs"),
+                (o_x, l_x, lambda r: orc.mask_vs_exact(r, w.N, gv[hi], gs[hi]), "vs exact"),
+                (o_bs, l_bs, lambda r: orc.mask_bs(r, w.N, gi[hi], gc[hi]), "bs"),
+                (o_a, l_a, lambda r: orc.mask_ashape(r, w.N, 16, 100), "a-shape"),
+                (o_d, l_d, lambda r: orc.mask_dense(r, w.N), "dense"),
+            ]
+            for o, l, mfn, name in cases:
+                O, L = orc.attention_head(qn[h], kn[kv], vn[kv], rows, mfn, sc)
+                check_close(o[bb, h].float().cpu().numpy(), O, f"b{bb} {name} h{h}")
+                check_lse(l[bb, h].cpu().numpy(), L, f"b{bb} {name} h{h}")
