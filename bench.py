@@ -132,6 +132,20 @@ def _recorded_traffic():
         return None
 
 
+def _patterns_text(w) -> str:
+    """Head -> pattern table of a workload, as text for the JSON line."""
+    from dynamic_sparse_attention_minf_b200 import workloads as wl
+    parts = []
+    nvs, nbs, na = (len(w.heads_of(p)) for p in (wl.PAT_VS, wl.PAT_BS, wl.PAT_A))
+    if nvs:
+        parts.append(f"{nvs} vertical-slash ({w.k_v}/{w.k_s})")
+    if nbs:
+        parts.append(f"{nbs} block-sparse (top-{w.k_b})")
+    if na:
+        parts.append(f"{na} a-shape ({w.n_sink}+{w.n_local})")
+    return ", ".join(parts)
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws > 1:
@@ -243,7 +257,7 @@ def run_reference(args, dist, rank, world):
     if rank != 0:
         return
     from dynamic_sparse_attention_minf_b200 import workloads as wl
-    w = wl.config(WORKLOAD_ID)
+    w = wl.config(args.config)
     q, k, v = wl.make_qkv(w, "cuda" if torch.cuda.is_available() else "cpu")
     times, flops_l, samples = [], [], []
     for step in range(args.warmup + args.steps):
@@ -274,7 +288,7 @@ def run_ours(args, dist, rank, world, local):
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = wl.config(WORKLOAD_ID)
+    w = wl.config(args.config)
     w.seed += 100 * rank                      # independent prompts per rank
     q, k, v = wl.make_qkv(w, dev)
     plan = layer.make_plan(w, dev)
@@ -282,14 +296,15 @@ def run_ours(args, dist, rank, world, local):
     stream = torch.cuda.current_stream(dev)
 
     # one counted run: executed tiles and kept entries per pattern
-    for name in ("ws_vs_attn", "ws_bs_attn", "ws_a"):
+    attn_ws = [n for n in ("ws_vs_attn", "ws_bs_attn", "ws_a") if n in plan.bufs]
+    for name in attn_ws:
         plan.bufs[name].zero_()
     layer.run_layer(plan, q, k, v, o)
     torch.cuda.synchronize()
     status = layer.device_status(plan)
     if status:
         raise RuntimeError(f"device status {status}")
-    cnt = {n: _counters(plan.bufs[n]) for n in ("ws_vs_attn", "ws_bs_attn", "ws_a")}
+    cnt = {n: _counters(plan.bufs[n]) for n in attn_ws}
     tile_flops = 4.0 * 128 * 128 * w.d
     useful = sum(4.0 * w.d * c[1] for c in cnt.values())
     executed = sum(tile_flops * c[0] for c in cnt.values())
@@ -423,9 +438,10 @@ def run_ours(args, dist, rank, world, local):
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-                   "patterns": "24 vertical-slash (2000/12000), 6 block-sparse (top-100), 2 a-shape (128+4096)",
+                   "patterns": _patterns_text(w),
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "inputs 12 GiB per step, larger than the 126 MB L2 (no flush needed)"},
+                   "l2": f"inputs {(q.numel() + k.numel() + v.numel()) * 2 / 2**30:.1f} GiB per step, larger than "
+                         "the 126 MB L2 (no flush needed)"},
         "step_ms_each": [round(x, 2) for x in per_step],
         "phase_ms": phase_ms,
         "useful_tflop_per_step": useful / 1e12, "executed_tflop_per_step": executed / 1e12,
@@ -488,6 +504,9 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense baseline")
     ap.add_argument("--no-exact", action="store_true", help="skip the element-exact VS variant")
+    ap.add_argument("--config", type=int, default=WORKLOAD_ID, choices=[2, 3, 4],
+                    help="workload: 4 (default) the 1M-token mixed layer, 2 the 128K mixed layer, "
+                         "3 the 512K all-Vertical-Slash layer")
     ap.add_argument("--kernel", choices=["dense", "vs"], default=None,
                     help="run only this attention kernel on a small case (for profiling)")
     ap.add_argument("--N", type=int, default=262144, help="tokens of the --kernel case")
