@@ -125,6 +125,17 @@ __device__ __forceinline__ uint64_t brev64(uint64_t x) {
 
 // A wait whose outcome is the same for every lane of the warp (the TMEM
 // accesses that follow are warp-collective).
+// True in exactly one lane of a fully active warp, the same lane every time.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(e));
+  return e != 0;
+}
+
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, DevStatus* st,
                                           int where) {
   const bool ok = mbar_wait(bar, parity, abort, st, where);
@@ -332,6 +343,7 @@ struct Producer {
     if (!acquire_k(stage)) return;
     if (lane == 0) {
       desc[stage].kind = KIND_END;
+      desc[stage].flags = 0;
       mbar_arrive(&k_full[stage]);
     }
     __syncwarp();
@@ -760,21 +772,23 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 8) {
     // --------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t qaddr = smem_u32(smem + C::kOffQ);
-      // O_0 += P[:, 0:64] V[0:64, :] and O_1 += P[:, 64:128] V[64:128, :];
-      // warpgroup w's bf16 P occupies TMEM columns 64w .. 64w+31 of the buffer
-      auto issue_pv = [&](int tp) -> bool {
-        const int bp = tp & 1;
-        const int sp = tp % C::kStages;
-        if (!mbar_wait(&p_full[bp], (tp >> 1) & 1, abort, p.status, 3)) return false;
-        if (!mbar_wait(&v_full[sp], (tp / C::kStages) & 1, abort, p.status, 4)) return false;
-        tc_fence_after();
-        // descriptors of the K-steps: the stage's base plus a constant (the
-        // start-address field holds address / 16 and never carries out)
-        const uint64_t vd0 = sdesc_sw128(smem_u32(smem + C::kOffV + sp * C::kKVBytes), C::kRegion, 1024);
-        const uint32_t a0 = tmem + bp * 128;
-        const uint32_t acc0 = tp > 0 ? 1u : 0u;
+    // The whole warp runs the loop, so that stage indices and descriptors are
+    // warp-uniform; one elected lane issues the MMAs and their commits.
+    const uint32_t qaddr = smem_u32(smem + C::kOffQ);
+    // O_0 += P[:, 0:64] V[0:64, :] and O_1 += P[:, 64:128] V[64:128, :];
+    // warpgroup w's bf16 P occupies TMEM columns 64w .. 64w+31 of the buffer
+    auto issue_pv = [&](int tp) -> bool {
+      const int bp = tp & 1;
+      const int sp = tp % C::kStages;
+      if (!warp_wait(&p_full[bp], (tp >> 1) & 1, abort, p.status, 3)) return false;
+      if (!warp_wait(&v_full[sp], (tp / C::kStages) & 1, abort, p.status, 4)) return false;
+      tc_fence_after();
+      // descriptors of the K-steps: the stage's base plus a constant (the
+      // start-address field holds address / 16 and never carries out)
+      const uint64_t vd0 = sdesc_sw128(smem_u32(smem + C::kOffV + sp * C::kKVBytes), C::kRegion, 1024);
+      const uint32_t a0 = tmem + bp * 128;
+      const uint32_t acc0 = tp > 0 ? 1u : 0u;
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t d_tmem = tmem + (kk < 4 ? C::kColO0 : C::kColO1);
@@ -782,20 +796,23 @@ __global__ void __launch_bounds__(320, 1)
                   (kk & 3) > 0 ? 1u : acc0);
         }
         umma_commit(&v_empty[sp]);
-        return true;
-      };
-      bool ok = mbar_wait(q_full, 0, abort, p.status, 2);
-      const uint64_t qd0 = sdesc_sw128(qaddr, 16, 1024);
-      int t = 0, pend = -1;
-      while (ok) {
-        const int st = t % C::kStages;
-        if (!mbar_wait(&k_full[st], (t / C::kStages) & 1, abort, p.status, 5)) { ok = false; break; }
-        if (desc[st].kind == KIND_END) break;
-        // Q and K were written by TMA or by cp.async plus the producer's proxy
-        // fence; the barrier alone orders them before the MMA (no tcgen05
-        // fence here: it would stall the issue of every tile).
-        const int w = t & 1;  // S buffer
-        const uint64_t kd0 = sdesc_sw128(smem_u32(smem + C::kOffK + st * C::kKVBytes), 16, 1024);
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = warp_wait(q_full, 0, abort, p.status, 2);
+    const uint64_t qd0 = sdesc_sw128(qaddr, 16, 1024);
+    int t = 0, pend = -1;
+    while (ok) {
+      const int st = t % C::kStages;
+      if (!warp_wait(&k_full[st], (t / C::kStages) & 1, abort, p.status, 5)) { ok = false; break; }
+      if (__all_sync(0xFFFFFFFFu, desc[st].kind == KIND_END)) break;
+      // Q and K were written by TMA or by cp.async plus the producer's proxy
+      // fence; the barrier alone orders them before the MMA (no tcgen05
+      // fence here: it would stall the issue of every tile).
+      const int w = t & 1;  // S buffer
+      const uint64_t kd0 = sdesc_sw128(smem_u32(smem + C::kOffK + st * C::kKVBytes), 16, 1024);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off16 = (uint64_t)(((kk >> 2) * C::kRegion + (kk & 3) * 32) / 16);
@@ -803,12 +820,16 @@ __global__ void __launch_bounds__(320, 1)
         }
         umma_commit(&s_full[w]);
         umma_commit(&k_empty[st]);
-        if (pend >= 0 && !issue_pv(pend)) { ok = false; pend = -1; break; }
-        pend = t;
-        ++t;
       }
-      if (ok && pend >= 0) issue_pv(pend);
-      umma_commit(mma_done);
+      __syncwarp();
+      if (pend >= 0 && !issue_pv(pend)) { ok = false; pend = -1; break; }
+      pend = t;
+      ++t;
+    }
+    if (ok && pend >= 0) issue_pv(pend);
+    if (elect_one()) umma_commit(mma_done);
+    __syncwarp();
+    if (lane == 0) {
       int dummy = 0;
       mbar_wait(mma_done, 0, &dummy, p.status, 7);
     }
@@ -829,12 +850,17 @@ __global__ void __launch_bounds__(320, 1)
       const int st = t % C::kStages;
       if (!warp_wait(&k_full[st], (t / C::kStages) & 1, abort, p.status, 10)) break;
       const TileDesc& dd = desc[st];
-      const int kind = dd.kind;
+      // kind and flags, rebuilt through one vote so that every test on them
+      // is warp-uniform for the compiler too (bit l of the word is lane l's)
+      const uint32_t kf = __ballot_sync(
+          0xFFFFFFFFu, ((((uint32_t)dd.kind & 0xFFu) << 8 | ((uint32_t)dd.flags & 0xFFu)) >> lane) & 1u);
+      const int kind = (int)(kf >> 8);
+      const int flags = (int)(kf & 0xFFu);
       if (kind == KIND_END) break;
       // element-exact tiles: the bitmap words of this row's window are
       // requested before waiting for the scores
       Window64 xs, xv;
-      const bool exact = POL == POL_VS_EXACT && (dd.flags & F_EXACT);
+      const bool exact = POL == POL_VS_EXACT && (flags & F_EXACT);
       if (exact) {
         const size_t hb = ((size_t)b * p.nh + hi) * p.bits_words;
         const int jw = dd.j0[wg];
@@ -843,7 +869,6 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (!warp_wait(&s_full[t & 1], (t >> 1) & 1, abort, p.status, 11)) break;
       tc_fence_after();
-      const int flags = dd.flags;
       const uint32_t scol = srow + (t & 1) * 128 + wg * 64;
       // Membership words of this warp's 64-row half for the warpgroup's two
       // 32-column chunks.  All rows of a warp lie in one half, so the chunk
@@ -857,13 +882,21 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (exact) {
         // bit c: (i - j in S) or (j in V) for key j = j0 + c; these words
-        // differ between rows, so the chunk tests below are per thread here
+        // differ between rows, so a chunk is skipped only if empty in all
         uint64_t em = brev64(xs.bits()) | xv.bits();
         // causal as bits: key j0 + c is allowed for c <= i - j0
         const int lim = i - dd.j0[wg];
         em &= (lim >= 63) ? ~0ull : (lim < 0 ? 0ull : ((2ull << lim) - 1ull));
         mw[0] &= (uint32_t)em;
         mw[1] &= (uint32_t)(em >> 32);
+      }
+      // chunk c2 needs no masking if full in every row, and no exponentials
+      // if empty in every row
+      bool cfull[2], cany[2];
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        cfull[c2] = __all_sync(0xFFFFFFFFu, mw[c2] == 0xFFFFFFFFu);
+        cany[c2] = __any_sync(0xFFFFFFFFu, mw[c2] != 0u);
       }
       uint32_t sr[2][32];
       tmem_ld32(scol, sr[0]);
@@ -876,7 +909,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
 #pragma unroll
       for (int c2 = 0; c2 < 2; ++c2) {
-        if (mw[c2] != 0xFFFFFFFFu && mw[c2] != 0u) {
+        if (!cfull[c2] && cany[c2]) {
 #pragma unroll
           for (int e = 0; e < 32; ++e)
             if (!((mw[c2] >> e) & 1u)) s[c2 * 32 + e] = -INFINITY;
@@ -903,7 +936,7 @@ __global__ void __launch_bounds__(320, 1)
         }
 #pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) {
-          if (mw[c2] != 0u) {
+          if (cany[c2]) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) nnz += (s[c2 * 32 + e] != -INFINITY);
           }
@@ -918,7 +951,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int k8 = 0; k8 < 8; ++k8) mx8[k8] = -INFINITY;
 #pragma unroll
       for (int c2 = 0; c2 < 2; ++c2) {
-        if (mw[c2] != 0u) {
+        if (cany[c2]) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[c2 * 32 + e]);
         }
@@ -940,7 +973,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int c2 = 0; c2 < 2; ++c2) {
         uint32_t pk[16];
-        if (mw[c2] != 0u) {
+        if (cany[c2]) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             float x0, x1;
