@@ -77,6 +77,23 @@ bool make_map(CUtensorMap* m, const void* ptr, long long rows, int d, int box_ro
   return r == CUDA_SUCCESS;
 }
 
+// 3-D bf16 view of a row-major [rows, d] matrix: x = column within a 64-column
+// region, y = row, z = region (global stride 128 B).  A box of 64 x box_rows x
+// d/64 lands region z at z * box_rows * 128 B in shared memory, each region
+// 128B-swizzled: the same layout as d/64 separate 2-D copies.
+bool make_map3(CUtensorMap* m, const void* ptr, long long rows, int d, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(d / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)(d / 64)};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 minf_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MINF_OK : MINF_ERR_CUDA; }
 
 // ----------------------------------------------------------- workspace plans
@@ -148,8 +165,8 @@ minf_status attn_launch(int pol, const minf_shape* s, const AttnParams& p, void*
   CUtensorMap tq, tk, tv, tk2, tv2;
   const long long kv_rows = (long long)s->B * s->Hkv * s->N;
   if (!make_map(&tq, p.Q, (long long)s->B * s->Hq * s->N, s->d, 128) || !make_map(&tk, p.K, kv_rows, s->d, 64) ||
-      !make_map(&tv, p.V, kv_rows, s->d, 64) || !make_map(&tk2, p.K, kv_rows, s->d, 128) ||
-      !make_map(&tv2, p.V, kv_rows, s->d, 128))
+      !make_map(&tv, p.V, kv_rows, s->d, 64) || !make_map3(&tk2, p.K, kv_rows, s->d, 128) ||
+      !make_map3(&tv2, p.V, kv_rows, s->d, 128))
     return MINF_ERR_CUDA;
   return cuda_status(attn_dispatch(s->d, pol, tq, tk, tv, tk2, tv2, p, (cudaStream_t)stream));
 }

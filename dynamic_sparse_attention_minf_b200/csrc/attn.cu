@@ -156,7 +156,7 @@ struct Producer {
   uint64_t* d_empty;
   const CUtensorMap* tmK;   // 64-row boxes
   const CUtensorMap* tmV;
-  const CUtensorMap* tmK2;  // 128-row boxes, for two adjacent chunks
+  const CUtensorMap* tmK2;  // 128-row boxes over all d/64 column regions (3-D view)
   const CUtensorMap* tmV2;
   const __nv_bfloat16* Kh;  // this (batch, kv head)'s K rows
   const __nv_bfloat16* Vh;
@@ -222,8 +222,7 @@ struct Producer {
       uint8_t* vb = smem + C::kOffV + stage * C::kKVBytes;
       mbar_arrive_expect_tx(&v_full[stage], C::kKVBytes);
       if (vj0[1] == vj0[0] + 64) {
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h) tma_load_2d(vb + h * C::kRegion, tmV2, &v_full[stage], 64 * h, kv_row0 + vj0[0]);
+        tma_load_3d(vb, tmV2, &v_full[stage], 0, kv_row0 + vj0[0], 0);
       } else {
 #pragma unroll
         for (int h = 0; h < D / 64; ++h) {
@@ -258,8 +257,7 @@ struct Producer {
       uint8_t* kb = smem + C::kOffK + stage * C::kKVBytes;
       mbar_arrive_expect_tx(&k_full[stage], C::kKVBytes);
       if (j0b == j0a + 64) {
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h) tma_load_2d(kb + h * C::kRegion, tmK2, &k_full[stage], 64 * h, kv_row0 + j0a);
+        tma_load_3d(kb, tmK2, &k_full[stage], 0, kv_row0 + j0a, 0);
       } else {
 #pragma unroll
         for (int h = 0; h < D / 64; ++h) {
