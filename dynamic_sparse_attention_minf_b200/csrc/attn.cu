@@ -859,15 +859,12 @@ __global__ void __launch_bounds__(320, 1)
       // requested before waiting for the scores
       Window64 xs, xv;
       const bool exact = POL == POL_VS_EXACT && (flags & F_EXACT);
+      const int jw = dd.j0[wg];  // RANGE tiles: first key of this warpgroup's chunk
       if (exact) {
         const size_t hb = ((size_t)b * p.nh + hi) * p.bits_words;
-        const int jw = dd.j0[wg];
         xs.load(p.sbits + hb, i - jw - 63);
         xv.load(p.vbits + hb, jw);
       }
-      if (!warp_wait(&s_full[t & 1], (t >> 1) & 1, abort, p.status, 11)) break;
-      tc_fence_after();
-      const uint32_t scol = srow + (t & 1) * 128 + wg * 64;
       // Membership words of this warp's 64-row half for the warpgroup's two
       // 32-column chunks.  All rows of a warp lie in one half, so the chunk
       // tests are warp-uniform: full chunks need no masking, empty chunks are
@@ -878,12 +875,18 @@ __global__ void __launch_bounds__(320, 1)
         mw[0] = m2.x;
         mw[1] = m2.y;
       }
+      // a RANGE descriptor is fully read: release it (and with it the K slot)
+      // before waiting for the scores; a GATHER one is read until the causal test
+      if (kind != KIND_GATHER) mbar_arrive(&d_empty[st]);
+      if (!warp_wait(&s_full[t & 1], (t >> 1) & 1, abort, p.status, 11)) break;
+      tc_fence_after();
+      const uint32_t scol = srow + (t & 1) * 128 + wg * 64;
       if (exact) {
         // bit c: (i - j in S) or (j in V) for key j = j0 + c; these words
         // differ between rows, so a chunk is skipped only if empty in all
         uint64_t em = brev64(xs.bits()) | xv.bits();
         // causal as bits: key j0 + c is allowed for c <= i - j0
-        const int lim = i - dd.j0[wg];
+        const int lim = i - jw;
         em &= (lim >= 63) ? ~0ull : (lim < 0 ? 0ull : ((2ull << lim) - 1ull));
         mw[0] &= (uint32_t)em;
         mw[1] &= (uint32_t)(em >> 32);
@@ -917,7 +920,6 @@ __global__ void __launch_bounds__(320, 1)
         const bool causal = flags & F_CAUSAL;
         const bool ash = flags & F_ASHAPE;
         if (kind == KIND_RANGE) {
-          const int jw = dd.j0[wg];
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
             const int j = jw + c;
@@ -942,7 +944,7 @@ __global__ void __launch_bounds__(320, 1)
       } else {
         nnz += __popc(mw[0]) + __popc(mw[1]);
       }
-      mbar_arrive(&d_empty[st]);  // descriptor no longer read
+      if (kind == KIND_GATHER) mbar_arrive(&d_empty[st]);  // descriptor no longer read
       // row max: eight independent chains over the non-empty chunks
       float mx8[8];
 #pragma unroll
