@@ -140,7 +140,7 @@ minf_status minf_estimate_vs(const minf_shape* shape, const minf_bf16* Q, const 
                              void* ws, size_t ws_bytes, void* stream);
 
 /*
- * Allocation-free variant of minf_estimate_vs.  The paper has no counterpart:
+ * Allocation-free variant of minf_estimate_vs.  MInference has no counterpart:
  * this exists for callers that cannot allocate device memory where they run
  * the estimation (for example code inside a CUDA-graph capture that forbids
  * allocation, or an engine plugin whose memory was planned up front), so they
