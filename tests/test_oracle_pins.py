@@ -417,3 +417,29 @@ def test_vs_exact_index_reproduces_mask(seed):
                 if j <= i:
                     got[i, j] = True
     assert np.array_equal(got, ref)
+
+
+# ------------------------------------------------- head map and conversion
+
+def test_kv_head_matches_repeat_interleave():
+    """GQA reading: expanding the KV heads with repeat_interleave (each KV head
+    serving g consecutive query heads, the LLaMA grouping) puts KV head
+    kv_head(h) at query head h."""
+    for Hq, Hkv in [(32, 8), (8, 2), (4, 4), (6, 1)]:
+        expanded = torch.arange(Hkv).repeat_interleave(Hq // Hkv)
+        assert [orc.kv_head(h, Hq, Hkv) for h in range(Hq)] == expanded.tolist()
+
+
+def test_to_f64_is_exact_bf16_decoding():
+    """bf16 -> float64 equals decoding the 16 stored bits by hand: sign,
+    8-bit exponent, 7-bit fraction, normal and subnormal."""
+    rng = np.random.default_rng(12)
+    bits = rng.integers(0, 1 << 16, 4096)
+    bits = bits[((bits >> 7) & 0xFF) != 0xFF]                 # no inf / nan encodings
+    x = torch.from_numpy(bits.astype(np.uint16).view(np.int16)).view(torch.bfloat16)
+    got = orc.to_f64(x)
+    for b, g in zip(bits.tolist(), got.tolist()):
+        sign = -1.0 if b >> 15 else 1.0
+        e, f = (b >> 7) & 0xFF, b & 0x7F
+        ref = sign * (f / 128.0 * 2.0 ** -126 if e == 0 else (1 + f / 128.0) * 2.0 ** (e - 127))
+        assert g == ref, (b, g, ref)
