@@ -3,14 +3,16 @@
 //
 //   warps 0-3  softmax warpgroup 0: key columns 0-63 of every tile  (thread = query row)
 //   warps 4-7  softmax warpgroup 1: key columns 64-127 of every tile
-//   warp  8    tcgen05 issuer (one lane) and TMEM owner
+//   warp  8    tcgen05 issuer (the whole warp runs the loop, one elected lane
+//              issues) and TMEM owner
 //   warp  9    producer: enumerates the key tiles of the query tile for the
 //              head's pattern, writes each tile's descriptor (column ids and
 //              per-64-row-half membership masks) and stages K and V into two
 //              rings of shared-memory slots: by TMA for contiguous 64-key
-//              chunks (one 128-row box when the two chunks are adjacent), by
-//              cp.async for gathered columns.  A K slot frees when S of its
-//              tile is done, a V slot when P V is; the V of a range tile is
+//              chunks (one 3-D copy of all column regions when the two chunks
+//              are adjacent), by cp.async for gathered columns.  A K slot frees
+//              when S of its tile is done and the softmax has released its
+//              descriptor, a V slot when P V is done; the V of a range tile is
 //              loaded after the next tile's K.
 //
 // Per key tile t (128 keys) the issuer computes S = Q K^T into TMEM buffer
