@@ -1,0 +1,49 @@
+"""Host-side pieces of the bench: the launch count it reports, the source
+digest that decides whether the recorded DRAM traffic still applies, and the
+committed launch-list summary that the count must agree with."""
+import os
+import re
+import types
+
+import bench
+from dynamic_sparse_attention_minf_b200 import layer
+from dynamic_sparse_attention_minf_b200 import workloads as wl
+
+
+def _plan(cid):
+    w = wl.config(cid)
+    present = lambda pat: (object() if w.heads_of(pat) else None)
+    return types.SimpleNamespace(w=w, vs_heads=present(wl.PAT_VS), bs_heads=present(wl.PAT_BS),
+                                 a_heads=present(wl.PAT_A))
+
+
+def test_launches_per_step_matches_launch_list_profile():
+    """The count the bench reports equals the kernels ncu listed per layer."""
+    n = layer.launches_per_step(_plan(4))
+    text = open(os.path.join(bench.ROOT, "profiles", "launches_llama3_8b_layer_n1m.md")).read()
+    per_layer = int(re.search(r"(\d+) launches per layer", text).group(1))
+    layers = 9
+    listed = sum(int(c) for c in re.findall(r"^\| `minf::[^|]*\| (\d+) \|", text, re.M))
+    assert n == per_layer == listed // layers
+    assert listed % layers == 0
+
+
+def test_launches_per_step_other_layers():
+    # 512K, Vertical-Slash heads only: estimation 4 + two 9-launch top-k, index 3, attention 1
+    assert layer.launches_per_step(_plan(3)) == 26
+    # 128K mixed layer: the same kernels as the 1M layer
+    assert layer.launches_per_step(_plan(2)) == 31
+
+
+def test_digest_ignores_comments_and_whitespace():
+    a = "int f(int x) { return x + 1; }  // one\n/* two */"
+    b = "int  f(int x)\n{\n  return x + 1;   /* another note */ }\n"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(a.replace("+ 1", "+ 2"))
+
+
+def test_recorded_traffic_gated_by_digest(monkeypatch):
+    t = bench._recorded_traffic()
+    assert t is None or t > 0
+    monkeypatch.setattr(bench, "kernel_sources_digest", lambda: "0" * 64)
+    assert bench._recorded_traffic() is None
