@@ -50,13 +50,18 @@ def _peaks():
 class ClockSampler:
     """nvidia-smi clock / throttle sampling during the timed region."""
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, path: str | None = None):
+        import tempfile
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        if path is None:
+            fd, path = tempfile.mkstemp(prefix=f"minf_clocks_{index}_", suffix=".csv")
+            os.close(fd)
+        self.path = path
 
     def __enter__(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        if os.path.dirname(self.path):
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
@@ -325,7 +330,8 @@ def run_ours(args, dist, rank, world, local):
             marks.append((name, e))
 
     mk = Marks()
-    with ClockSampler(local) as clk:
+    clock_log = args.clock_log.replace("{rank}", str(rank)) if args.clock_log else None
+    with ClockSampler(local, clock_log) as clk:
         time.sleep(1.0)                      # let the sampler start before timing
         _barrier(dist)
         torch.cuda.synchronize()
@@ -510,6 +516,9 @@ def main():
     ap.add_argument("--kernel", choices=["dense", "vs"], default=None,
                     help="run only this attention kernel on a small case (for profiling)")
     ap.add_argument("--N", type=int, default=262144, help="tokens of the --kernel case")
+    ap.add_argument("--clock-log", default=None,
+                    help="keep the nvidia-smi clock samples in this CSV file ({rank} is replaced by the "
+                         "rank); default: a temporary file")
     args = ap.parse_args()
     if args.kernel:
         run_kernel_case(args)

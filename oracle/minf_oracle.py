@@ -186,8 +186,14 @@ def bs_select(q: np.ndarray, k: np.ndarray, scale: float, k_b: int, block: int =
     change the selection.  Returns idx [nb, k_b] (ascending, -1 padded) and
     cnt [nb] = min(b + 1, k_b).  With ``blocks`` given, only those query
     blocks are selected (rows of the result follow ``blocks``)."""
-    qbar = bs_pool(q, block)
-    kbar = bs_pool(k, block)
+    return bs_select_pooled(bs_pool(q, block), bs_pool(k, block), scale, k_b, blocks)
+
+
+def bs_select_pooled(qbar: np.ndarray, kbar: np.ndarray, scale: float, k_b: int, blocks=None):
+    """The selection of :func:`bs_select` from already pooled queries and
+    keys (``qbar``, ``kbar``: [nb, d]).  Row r of the result is query block
+    ``blocks[r]`` (every block when ``blocks`` is None): its candidates are
+    the key blocks c <= blocks[r], and c = blocks[r] is forced."""
     nb = qbar.shape[0]
     b = np.arange(nb) if blocks is None else np.asarray(blocks, np.int64)
     t = bs_scores(qbar[b], kbar, scale)

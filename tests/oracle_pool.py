@@ -144,9 +144,8 @@ def check_head(task: dict) -> dict:
             step = 512
             for b0 in range(0, nb, step):
                 b = np.arange(b0, min(nb, b0 + step))
-                t = orc.bs_scores(qbar[b], kbar, sc)
-                valid = np.arange(nb)[None, :] <= b[:, None]
-                ri, rc = orc.select_topk_rows(t, valid, task["k_b"], forced_col=b)
+                ri, rc = orc.bs_select_pooled(qbar, kbar, sc, task["k_b"], blocks=b)
+                t = orc.bs_scores(qbar[b], kbar, sc)      # the scores the gap rule reads
                 if not np.array_equal(rc, gc[b]):
                     out["errors"].append(f"blk_cnt differs near block {b0}")
                     break

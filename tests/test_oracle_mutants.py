@@ -100,6 +100,22 @@ def _bs_select_no_forced(q, k, scale, k_b, block=64, blocks=None):
     return orc.select_topk_rows(t, valid, k_b, forced_col=None)
 
 
+def _bs_select_pooled_rows_by_position(qbar, kbar, scale, k_b, blocks=None):
+    nb = qbar.shape[0]
+    b = np.arange(nb) if blocks is None else np.asarray(blocks, np.int64)
+    t = orc.bs_scores(qbar[b], kbar, scale)
+    valid = np.arange(nb)[None, :] <= np.arange(len(b))[:, None]      # row position, not block id
+    return orc.select_topk_rows(t, valid, k_b, forced_col=b)
+
+
+def _bs_select_pooled_forced_by_position(qbar, kbar, scale, k_b, blocks=None):
+    nb = qbar.shape[0]
+    b = np.arange(nb) if blocks is None else np.asarray(blocks, np.int64)
+    t = orc.bs_scores(qbar[b], kbar, scale)
+    valid = np.arange(nb)[None, :] <= b[:, None]
+    return orc.select_topk_rows(t, valid, k_b, forced_col=np.arange(len(b)))   # not following blocks
+
+
 def _vs_groups_strict(s_idx, block=64):
     s = np.asarray(s_idx, np.int64)
     if s.size == 0:
@@ -210,6 +226,9 @@ MUTANTS = {
         "bs_pool": lambda x, block=64: _ORIG["bs_pool"](x, block) * block},
     "bs_scores: operands transposed": {"bs_scores": lambda qb, kb, sc: sc * (kb @ qb.T)},
     "bs_select: diagonal block not forced": {"bs_select": _bs_select_no_forced},
+    "bs_select_pooled: causal limit from the row position": {"bs_select_pooled": _bs_select_pooled_rows_by_position},
+    "bs_select_pooled: forced block from the row position": {
+        "bs_select_pooled": _bs_select_pooled_forced_by_position},
     "vs_groups: offsets exactly 64 apart not merged": {"vs_groups": _vs_groups_strict},
     "vs_block_verticals: verticals inside bands kept": {"vs_block_verticals": _vs_block_verticals_no_dedup},
     "mask_vs: band one key too wide": {

@@ -295,6 +295,31 @@ def test_bs_select_all_blocks_closed_form():
         assert cnt[b] == b + 1 and idx[b, : b + 1].tolist() == list(range(b + 1))
 
 
+def test_bs_select_subset_of_blocks_bruteforce_loops():
+    """Selection restricted to a subset of query blocks (given out of order,
+    not contiguous), against plain loops: pooled means, scores for c <= b,
+    diagonal forced, ranked by (score desc, index asc), first k ascending."""
+    rng = np.random.default_rng(12)
+    nb, d, k_b = 12, 6, 4
+    q = rng.standard_normal((64 * nb, d))
+    k = rng.standard_normal((64 * nb, d))
+    blocks = [9, 2, 11, 5, 0, 7]
+    sc = 0.7
+    idx, cnt = orc.bs_select(q, k, sc, k_b, blocks=blocks)
+    idx_p, cnt_p = orc.bs_select_pooled(orc.bs_pool(q), orc.bs_pool(k), sc, k_b, blocks=blocks)
+    assert np.array_equal(idx, idx_p) and np.array_equal(cnt, cnt_p)
+    mean = lambda x, b, t: sum(x[64 * b + r, t] for r in range(64)) / 64
+    for row, b in enumerate(blocks):
+        cand = []
+        for c in range(b + 1):
+            s = sc * sum(mean(q, b, t) * mean(k, c, t) for t in range(d))
+            cand.append((-math.inf if c == b else -s, c))
+        chosen = sorted(c for _, c in sorted(cand)[: min(k_b, b + 1)])
+        assert cnt[row] == len(chosen)
+        assert idx[row, : cnt[row]].tolist() == chosen, (b, idx[row], chosen)
+        assert (idx[row, cnt[row]:] == -1).all()
+
+
 # ------------------------------------------------------ VS index build
 
 def test_vs_groups_loops():
