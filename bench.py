@@ -14,8 +14,12 @@ the tiles it actually executes.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-With N > 1 (torchrun) every rank runs its own layer (independent prompts, no
-collective on the data path: weak scaling); time is the max over ranks.
+With N > 1 (torchrun) the layer is split across the ranks by KV-head group
+(``--shard kv``, the default): rank r computes the query heads of KV heads
+[r Hkv/N, (r+1) Hkv/N) with their rows of the pattern table, O stays
+head-sharded and no collective touches the data path (strong scaling).
+``--shard replicas`` runs one independent layer per rank instead (weak
+scaling).  Time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -101,7 +105,7 @@ class ClockSampler:
 
 
 _KERNEL_SOURCES = ("csrc/attn.cu", "csrc/minf_device.cuh", "csrc/minf_internal.h")
-_TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "attn_vs_llama3_8b_layer_n1m_dram.md")
+_TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "attn_vs_n256k_dram.md")
 
 
 def _code_only(src: str) -> str:
@@ -123,16 +127,18 @@ def kernel_sources_digest() -> str:
 
 
 def _recorded_traffic():
-    """DRAM bytes (read + write) of one Vertical-Slash attention launch of the
-    1M layer, from the committed ncu summary, or None when the attention
-    sources no longer hash to the ones that summary was captured from."""
+    """DRAM bytes (read + write) per executed 128 x 128 tile of the attention
+    kernel, from the committed ncu summary of one Vertical-Slash launch at
+    256K tokens (8 query / 2 KV heads), or None when the attention sources no
+    longer hash to the ones that summary was captured from.  The bench scales
+    it by the executed tiles of the launch it reports."""
     try:
         text = open(_TRAFFIC_PROFILE).read()
         vals = dict(line.split(": ", 1) for line in text.splitlines()
-                    if line.startswith(("traffic_bytes_per_launch: ", "kernel_sources_sha256: ")))
+                    if line.startswith(("traffic_bytes_per_tile: ", "kernel_sources_sha256: ")))
         if vals.get("kernel_sources_sha256", "").strip() != kernel_sources_digest():
             return None
-        return float(vals["traffic_bytes_per_launch"])
+        return float(vals["traffic_bytes_per_tile"])
     except (OSError, KeyError, ValueError):
         return None
 
@@ -176,8 +182,18 @@ def _max_over_ranks(dist, x: float) -> float:
 
 
 def _throughput(world: int, flops_per_rank: float, ms: float) -> float:
-    """Whole-job TFLOP/s: every rank processes its own layer (weak scaling)."""
+    """Whole-job TFLOP/s when every rank processes its own layer (weak scaling)."""
     return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
+def _sum_over_ranks(dist, x: float) -> float:
+    """Sum of a per-rank quantity (every rank gets it)."""
+    if dist is None:
+        return x
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
 
 
 def _barrier(dist):
@@ -293,41 +309,70 @@ def run_ours(args, dist, rank, world, local):
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = wl.config(args.config)
-    w.seed += 100 * rank                      # independent prompts per rank
-    q, k, v = wl.make_qkv(w, dev)
+    w_full = wl.config(args.config)
+    shard = world > 1 and args.shard == "kv"
+    if shard:
+        # one layer split by KV-head group: every rank draws the same inputs
+        # and keeps its own heads
+        hq0, hq1, hk0, hk1 = layer.kv_group_slice(w_full, rank, world)
+        qf, kf, vf = wl.make_qkv(w_full, dev)
+        q, k, v = (x[:, a:b].contiguous() for x, a, b in ((qf, hq0, hq1), (kf, hk0, hk1), (vf, hk0, hk1)))
+        del qf, kf, vf
+        torch.cuda.empty_cache()
+        w = layer.local_workload(w_full, rank, world)
+    else:
+        w = w_full
+        w.seed += 100 * rank                  # independent prompts per rank
+        q, k, v = wl.make_qkv(w, dev)
     plan = layer.make_plan(w, dev)
     o = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
 
-    # one counted run: executed tiles and kept entries per pattern
+    # one counted run per pattern (one attention launch each): executed
+    # tiles and kept entries of every pattern; then the same layer with one
+    # attention launch for all heads, whose counters must add up to them
     attn_ws = [n for n in ("ws_vs_attn", "ws_bs_attn", "ws_a") if n in plan.bufs]
-    for name in attn_ws:
+    for name in attn_ws + ["ws_attn"]:
         plan.bufs[name].zero_()
-    layer.run_layer(plan, q, k, v, o)
+    layer.run_layer(plan, q, k, v, o, fused=False)
+    layer.run_layer(plan, q, k, v, o, fused=True)
     torch.cuda.synchronize()
     status = layer.device_status(plan)
     if status:
         raise RuntimeError(f"device status {status}")
     cnt = {n: _counters(plan.bufs[n]) for n in attn_ws}
+    fused_cnt = _counters(plan.bufs["ws_attn"])
     tile_flops = 4.0 * 128 * 128 * w.d
     useful = sum(4.0 * w.d * c[1] for c in cnt.values())
     executed = sum(tile_flops * c[0] for c in cnt.values())
-    vs_exec = tile_flops * cnt["ws_vs_attn"][0]
+    exec_tiles = sum(c[0] for c in cnt.values())
+    if fused_cnt != (exec_tiles, sum(c[1] for c in cnt.values())):
+        raise RuntimeError(f"one-launch counters {fused_cnt} differ from the per-pattern launches {cnt}")
 
     # warm-up
     for _ in range(args.warmup):
         layer.run_layer(plan, q, k, v, o)
     torch.cuda.synchronize()
 
-    # timed device steps, with events around the VS attention launch
+    # timed device steps, with events around every call of the layer
     marks = []
 
     class Marks:
+        def __init__(self):
+            self.events = []
+
         def mark(self, name):
             e = torch.cuda.Event(enable_timing=True)
             e.record(stream)
-            marks.append((name, e))
+            self.events.append((name, e))
+
+    def phase_means(events):
+        phases = {}
+        for a_, b_ in zip(events[0::2], events[1::2]):
+            name = a_[0].split(":")[0]
+            assert a_[0] == name + ":pre" and b_[0] == name + ":post"
+            phases.setdefault(name, []).append(a_[1].elapsed_time(b_[1]))
+        return {n: round(statistics.mean(t), 3) for n, t in phases.items()}
 
     mk = Marks()
     clock_log = args.clock_log.replace("{rank}", str(rank)) if args.clock_log else None
@@ -345,13 +390,17 @@ def run_ours(args, dist, rank, world, local):
     per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     step_ms = ev[0].elapsed_time(ev[-1]) / args.steps
     step_ms = _max_over_ranks(dist, step_ms)
-    phases = {}
-    for a, b in zip(marks[0::2], marks[1::2]):
-        name = a[0].split(":")[0]
-        assert a[0] == name + ":pre" and b[0] == name + ":post"
-        phases.setdefault(name, []).append(a[1].elapsed_time(b[1]))
-    phase_ms = {n: round(statistics.mean(t), 3) for n, t in phases.items()}
-    vs_ms = phase_ms.get("vs_attn")
+    phase_ms = phase_means(mk.events)
+    attn_ms = phase_ms.get("attn")
+
+    # the same layer with one attention launch per pattern, for comparison
+    # (outside the timed steps)
+    mk_sep = Marks()
+    for _ in range(2):
+        layer.run_layer(plan, q, k, v, o, marks=mk_sep, fused=False)
+    torch.cuda.synchronize()
+    sep_ms = phase_means(mk_sep.events)
+    attn_sep = {n: sep_ms[n] for n in ("vs_attn", "bs_attn", "a_attn") if n in sep_ms}
 
     # end to end through the public API: pinned host in, host out
     hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
@@ -422,14 +471,18 @@ def run_ours(args, dist, rank, world, local):
             "executed_tflops": tile_flops * x_tiles / (x_ms * 1e-3) / 1e12,
             "useful_tflops": 4.0 * w.d * x_nnz / (x_ms * 1e-3) / 1e12,
             "band_useful_tflop": 4.0 * w.d * cnt["ws_vs_attn"][1] / 1e12,
+            "band_tiles": cnt["ws_vs_attn"][0], "band_ms": attn_sep.get("vs_attn"),
         }
         del xi
 
+    # whole-job work: the ranks' shares of one layer add up (KV-head split),
+    # or every rank runs a layer of its own (replicas)
+    useful_job = _sum_over_ranks(dist, useful) if shard else world * useful
     if rank != 0:
         return
     peaks, src = _peaks()
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    achieved = vs_exec / (vs_ms * 1e-3) / 1e12 if vs_ms else None
+    achieved = executed / (attn_ms * 1e-3) / 1e12 if attn_ms else None
     cpu = None
     if world == 1 and not args.no_cpu:
         flops_c, total_s, sample_s, _ = oracle_sample(w, q, k, v, plan, rows_per_pattern=96)
@@ -437,31 +490,45 @@ def run_ours(args, dist, rank, world, local):
                "sample": "one head of each pattern with full index estimation and 96 sampled query rows, "
                          f"scaled to all heads and rows ({sample_s:.1f} s of CPU)"}
     clocks = clk.summary()
-    val = _throughput(world, useful, step_ms)
+    val = useful_job / (step_ms * 1e-3) / 1e12
     dense_flops = 4.0 * w.d * (w.N * (w.N + 1) / 2) * w.Hq
+    traffic = _recorded_traffic()
+    # tensor-pipe utilisation at the run's own clock: the bf16 MMA of this
+    # kernel (M = N = 128, K = 16) retires 8192 FLOP per clock per SM
+    sm_mhz = (clocks or {}).get("sm_mhz")
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    tensor_at_clock = (achieved / (8192.0 * nsm * sm_mhz * 1e6 / 1e12)) if (achieved and sm_mhz) else None
     line = {
         "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "strong" if shard else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-                   "patterns": _patterns_text(w),
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"inputs {(q.numel() + k.numel() + v.numel()) * 2 / 2**30:.1f} GiB per step, larger than "
-                         "the 126 MB L2 (no flush needed)"},
+        "config": {"workload": w_full.name, "N": w.N, "Hq": w_full.Hq, "Hkv": w_full.Hkv, "d": w.d,
+                   "patterns": _patterns_text(w_full),
+                   "parallelism": (f"kv-head groups x{world}" if shard else f"replicas{world}") if world > 1
+                   else "single",
+                   "l2": f"inputs {(q.numel() + k.numel() + v.numel()) * 2 / 2**30:.1f} GiB per step and rank, "
+                         "larger than the 126 MB L2 (no flush needed)"},
         "step_ms_each": [round(x, 2) for x in per_step],
         "phase_ms": phase_ms,
-        "useful_tflop_per_step": useful / 1e12, "executed_tflop_per_step": executed / 1e12,
+        "attn_ms_one_launch_per_pattern": attn_sep,
+        "useful_tflop_per_step": useful_job / 1e12, "executed_tflop_per_step": executed / 1e12,
         "density_vs_dense": useful / dense_flops,
         "dense_attn_ms_est": dense_ms,
         "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None,
-        "roofline": {"kernel": "attn_kernel<128, vertical_slash>", "bound": "tensor",
+        "roofline": {"kernel": f"attn_kernel<{w.d}> (one launch, every head of the layer)", "bound": "tensor",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": (achieved / peak) if achieved else None,
-                     "traffic": (_recorded_traffic() if w.N == 1 << 20 else None),
-                     "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
-                     "peak_source": f"{src} bf16_tflops_sustained", "ms_per_launch": vs_ms,
-                     "executed_tflop_per_launch": vs_exec / 1e12},
-        "e2e": {"value": _throughput(world, useful, e2e_ms), "unit": "TFLOP/s",
+                     "traffic": (traffic * exec_tiles) if traffic else None,
+                     "traffic_unit": "bytes per launch: ncu dram__bytes_read.sum + dram__bytes_write.sum per "
+                                     "executed tile of the 256K Vertical-Slash capture, times this launch's tiles",
+                     "peak_source": f"{src} bf16_tflops_sustained (of measured)" if src == "measured"
+                                    else f"{src} (of fallback)",
+                     "ms_per_launch": attn_ms, "executed_tflop_per_launch": executed / 1e12,
+                     "tensor_active_at_run_clock": tensor_at_clock,
+                     "vs_launch": {"tiles": cnt["ws_vs_attn"][0] if "ws_vs_attn" in cnt else None,
+                                   "ms_one_launch_per_pattern": attn_sep.get("vs_attn")}},
+        "e2e": {"value": useful_job / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "steps": e2e_steps,
                 "mode": "layer.run_pipelined: every step uploads its Q/K/V from pinned host memory and "
@@ -498,7 +565,14 @@ def run_kernel_case(args):
     for _ in range(args.warmup + args.steps):
         fn()
     torch.cuda.synchronize()
-    print(json.dumps({"kernel": args.kernel, "N": args.N, "launches": args.warmup + args.steps}))
+    # executed tiles of one launch (the device counter of a fresh workspace)
+    ws_k = b["ws_vs_attn"] if args.kernel == "vs" else ws
+    ws_k.zero_()
+    fn()
+    torch.cuda.synchronize()
+    tiles = _counters(ws_k)[0]
+    print(json.dumps({"kernel": args.kernel, "N": args.N, "launches": args.warmup + args.steps + 1,
+                      "tiles_per_launch": tiles, "kernel_sources_sha256": kernel_sources_digest()}))
 
 
 def main():
@@ -516,6 +590,8 @@ def main():
     ap.add_argument("--kernel", choices=["dense", "vs"], default=None,
                     help="run only this attention kernel on a small case (for profiling)")
     ap.add_argument("--N", type=int, default=262144, help="tokens of the --kernel case")
+    ap.add_argument("--shard", choices=["kv", "replicas"], default="kv",
+                    help="with several GPUs: split one layer by KV-head group (default) or run a layer per rank")
     ap.add_argument("--clock-log", default=None,
                     help="keep the nvidia-smi clock samples in this CSV file ({rank} is replaced by the "
                          "rank); default: a temporary file")

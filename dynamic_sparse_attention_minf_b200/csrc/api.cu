@@ -1,6 +1,7 @@
 // Host side of the libminf C ABI: argument validation, workspace carving,
 // TMA descriptor set-up and kernel dispatch.  See include/minf.h for the
 // contract of every entry point.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -135,22 +136,21 @@ size_t plan_bs_est(const minf_shape* s, int nh, char* ws, BsEstWs* out) {
   return c.off;
 }
 
-minf_status attn_common(int pol, const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
-                        const int32_t* heads, int nh, minf_bf16* O, float* lse, void* ws, size_t ws_bytes,
-                        void* stream, AttnParams& p) {
+// Checks the arguments every attention call shares and fills the common
+// part of the launch parameters (no segment yet).
+minf_status attn_common(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
+                        minf_bf16* O, float* lse, void* ws, size_t ws_bytes, AttnParams& p) {
   minf_status st = check_shape(s);
   if (st != MINF_OK) return st;
   if (!Q || !K || !V || !O || !ws) return MINF_ERR_INVALID_ARG;
-  if (nh < 1 || nh > s->Hq || (!heads && pol != POL_DENSE)) return MINF_ERR_INVALID_ARG;
   if (ws_bytes < kStatusBytes) return MINF_ERR_WORKSPACE_TOO_SMALL;
   if (((uintptr_t)Q | (uintptr_t)K | (uintptr_t)V | (uintptr_t)O) & 15) return MINF_ERR_INVALID_ARG;
+  std::memset(&p, 0, sizeof(p));
   p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
   p.K = reinterpret_cast<const __nv_bfloat16*>(K);
   p.V = reinterpret_cast<const __nv_bfloat16*>(V);
   p.O = reinterpret_cast<__nv_bfloat16*>(O);
   p.lse = lse;
-  p.heads = heads;
-  p.nh = heads ? nh : s->Hq;
   p.B = s->B;
   p.Hq = s->Hq;
   p.Hkv = s->Hkv;
@@ -161,14 +161,45 @@ minf_status attn_common(int pol, const minf_shape* s, const minf_bf16* Q, const 
   return MINF_OK;
 }
 
-minf_status attn_launch(int pol, const minf_shape* s, const AttnParams& p, void* stream) {
+// Appends a pattern's heads (heads == NULL means heads 0 .. nh-1).
+minf_status add_seg(AttnParams& p, int pol, const int32_t* heads, int nh) {
+  if (nh < 1 || nh > p.Hq || p.nseg >= 3) return MINF_ERR_INVALID_ARG;
+  p.seg[p.nseg].pol = pol;
+  p.seg[p.nseg].heads = heads;
+  p.seg[p.nseg].nh = nh;
+  ++p.nseg;
+  p.nh_total += nh;
+  return p.nh_total <= p.Hq ? MINF_OK : MINF_ERR_INVALID_ARG;
+}
+
+minf_status attn_launch(const minf_shape* s, AttnParams& p, void* stream) {
+  if (p.nseg < 1) return MINF_ERR_INVALID_ARG;
+  p.nqt = s->N / 128;
+  const long long items = (long long)p.nqt * s->B * p.nh_total;
+  if (items >= (1ll << 31)) return MINF_ERR_UNSUPPORTED;
+  p.nitems = (int)items;
   CUtensorMap tq, tk, tv, tk2, tv2;
   const long long kv_rows = (long long)s->B * s->Hkv * s->N;
   if (!make_map(&tq, p.Q, (long long)s->B * s->Hq * s->N, s->d, 128) || !make_map(&tk, p.K, kv_rows, s->d, 64) ||
       !make_map(&tv, p.V, kv_rows, s->d, 64) || !make_map3(&tk2, p.K, kv_rows, s->d, 128) ||
       !make_map3(&tv2, p.V, kv_rows, s->d, 128))
     return MINF_ERR_CUDA;
-  return cuda_status(attn_dispatch(s->d, pol, tq, tk, tv, tk2, tv2, p, (cudaStream_t)stream));
+  return cuda_status(attn_dispatch(s->d, tq, tk, tv, tk2, tv2, p, (cudaStream_t)stream));
+}
+
+bool vs_index_ok(const minf_vs_index* idx) {
+  return idx && idx->tgrp && idx->tgrp_cnt && idx->wmap && idx->vcnt && idx->vidx;
+}
+
+void set_vs_index(AttnParams& p, const minf_shape* s, const minf_vs_index* idx, int k_v, int k_s) {
+  p.tgrp = idx->tgrp;
+  p.tgrp_cnt = idx->tgrp_cnt;
+  p.wmap = idx->wmap;
+  p.vcnt = idx->vcnt;
+  p.vidx = idx->vidx;
+  p.k_s = k_s;
+  p.k_v = k_v;
+  p.wmap_words = (int)minf_vs_wmap_words(s->N);
 }
 
 }  // namespace
@@ -196,6 +227,7 @@ size_t minf_workspace_size(int op, const minf_shape* s, int nh, int k_v, int k_s
     case MINF_OP_SPARSE_ATTN_BS:
     case MINF_OP_ATTN_ASHAPE:
     case MINF_OP_DENSE_ATTN:
+    case MINF_OP_SPARSE_ATTN_LAYER:
       return kStatusBytes;
     default:
       return 0;
@@ -361,80 +393,108 @@ minf_status minf_sparse_attn_vs_exact(const minf_shape* s, const minf_bf16* Q, c
                                       const minf_vs_exact_index* idx, int k_v, int k_s, minf_bf16* O, float* lse,
                                       void* ws, size_t ws_bytes, void* stream) {
   AttnParams p;
-  std::memset(&p, 0, sizeof(p));
-  minf_status st = attn_common(POL_VS_EXACT, s, Q, K, V, heads, nh, O, lse, ws, ws_bytes, stream, p);
+  minf_status st = attn_common(s, Q, K, V, O, lse, ws, ws_bytes, p);
   if (st != MINF_OK) return st;
-  if (!idx || !idx->tgrp || !idx->tgrp_cnt || !idx->sbits || !idx->vbits || !idx->vcnt || !idx->vidx)
+  if (!heads || (st = add_seg(p, POL_VS_EXACT, heads, nh)) != MINF_OK) return MINF_ERR_INVALID_ARG;
+  if (!idx || !idx->tgrp || !idx->tgrp_cnt || !idx->sbits || !idx->vbits || !idx->twmap || !idx->vcnt ||
+      !idx->vidx)
     return MINF_ERR_INVALID_ARG;
   if (k_v < 1 || k_s < 1 || k_v > s->N || k_s > s->N) return MINF_ERR_INVALID_ARG;
   p.tgrp = idx->tgrp;
   p.tgrp_cnt = idx->tgrp_cnt;
   p.sbits = idx->sbits;
   p.vbits = idx->vbits;
+  p.twmap = idx->twmap;
   p.bits_words = (int)minf_vs_bits_words(s->N);
+  p.twmap_words = (int)minf_vs_twmap_words(s->N);  // unused by the kernel; kept with the index
   p.vcnt = idx->vcnt;
   p.vidx = idx->vidx;
   p.k_s = k_s;
   p.k_v = k_v;
-  return attn_launch(POL_VS_EXACT, s, p, stream);
+  return attn_launch(s, p, stream);
 }
 
 minf_status minf_sparse_attn_vs(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
                                 const int32_t* heads, int nh, const minf_vs_index* idx, int k_v, int k_s,
                                 minf_bf16* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
   AttnParams p;
-  std::memset(&p, 0, sizeof(p));
-  minf_status st = attn_common(POL_VS, s, Q, K, V, heads, nh, O, lse, ws, ws_bytes, stream, p);
+  minf_status st = attn_common(s, Q, K, V, O, lse, ws, ws_bytes, p);
   if (st != MINF_OK) return st;
-  if (!idx || !idx->tgrp || !idx->tgrp_cnt || !idx->wmap || !idx->vcnt || !idx->vidx) return MINF_ERR_INVALID_ARG;
+  if (!heads || add_seg(p, POL_VS, heads, nh) != MINF_OK) return MINF_ERR_INVALID_ARG;
+  if (!vs_index_ok(idx)) return MINF_ERR_INVALID_ARG;
   if (k_v < 1 || k_s < 1 || k_v > s->N || k_s > s->N) return MINF_ERR_INVALID_ARG;
-  p.tgrp = idx->tgrp;
-  p.tgrp_cnt = idx->tgrp_cnt;
-  p.wmap = idx->wmap;
-  p.vcnt = idx->vcnt;
-  p.vidx = idx->vidx;
-  p.k_s = k_s;
-  p.k_v = k_v;
-  p.wmap_words = (int)minf_vs_wmap_words(s->N);
-  return attn_launch(POL_VS, s, p, stream);
+  set_vs_index(p, s, idx, k_v, k_s);
+  return attn_launch(s, p, stream);
 }
 
 minf_status minf_sparse_attn_bs(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
                                 const int32_t* heads, int nh, const int32_t* blk_idx, const int32_t* blk_cnt,
                                 int k_b, minf_bf16* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
   AttnParams p;
-  std::memset(&p, 0, sizeof(p));
-  minf_status st = attn_common(POL_BS, s, Q, K, V, heads, nh, O, lse, ws, ws_bytes, stream, p);
+  minf_status st = attn_common(s, Q, K, V, O, lse, ws, ws_bytes, p);
   if (st != MINF_OK) return st;
+  if (!heads || add_seg(p, POL_BS, heads, nh) != MINF_OK) return MINF_ERR_INVALID_ARG;
   if (!blk_idx || !blk_cnt || k_b < 1) return MINF_ERR_INVALID_ARG;
   p.blk_idx = blk_idx;
   p.blk_cnt = blk_cnt;
   p.k_b = k_b;
-  return attn_launch(POL_BS, s, p, stream);
+  return attn_launch(s, p, stream);
 }
 
 minf_status minf_attn_ashape(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
                              const int32_t* heads, int nh, int n_sink, int n_local, minf_bf16* O, float* lse,
                              void* ws, size_t ws_bytes, void* stream) {
   AttnParams p;
-  std::memset(&p, 0, sizeof(p));
-  minf_status st = attn_common(POL_ASHAPE, s, Q, K, V, heads, nh, O, lse, ws, ws_bytes, stream, p);
+  minf_status st = attn_common(s, Q, K, V, O, lse, ws, ws_bytes, p);
   if (st != MINF_OK) return st;
+  if (!heads || add_seg(p, POL_ASHAPE, heads, nh) != MINF_OK) return MINF_ERR_INVALID_ARG;
   if (n_sink < 0 || n_local < 1) return MINF_ERR_INVALID_ARG;
   p.n_sink = n_sink;
   p.n_local = n_local;
-  return attn_launch(POL_ASHAPE, s, p, stream);
+  return attn_launch(s, p, stream);
 }
 
 minf_status minf_dense_attn(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
                             const int32_t* heads, int nh, minf_bf16* O, float* lse, void* ws, size_t ws_bytes,
                             void* stream) {
   AttnParams p;
-  std::memset(&p, 0, sizeof(p));
-  if (!heads && s && nh != s->Hq) nh = s->Hq;
-  minf_status st = attn_common(POL_DENSE, s, Q, K, V, heads, nh, O, lse, ws, ws_bytes, stream, p);
+  minf_status st = attn_common(s, Q, K, V, O, lse, ws, ws_bytes, p);
   if (st != MINF_OK) return st;
-  return attn_launch(POL_DENSE, s, p, stream);
+  if (!heads) nh = s->Hq;
+  if (add_seg(p, POL_DENSE, heads, nh) != MINF_OK) return MINF_ERR_INVALID_ARG;
+  return attn_launch(s, p, stream);
+}
+
+minf_status minf_sparse_attn_layer(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K,
+                                   const minf_bf16* V, const int32_t* vs_heads, int n_vs,
+                                   const minf_vs_index* vs_idx, int k_v, int k_s, const int32_t* bs_heads,
+                                   int n_bs, const int32_t* blk_idx, const int32_t* blk_cnt, int k_b,
+                                   const int32_t* a_heads, int n_a, int n_sink, int n_local, minf_bf16* O,
+                                   float* lse, void* ws, size_t ws_bytes, void* stream) {
+  AttnParams p;
+  minf_status st = attn_common(s, Q, K, V, O, lse, ws, ws_bytes, p);
+  if (st != MINF_OK) return st;
+  if (n_vs < 0 || n_bs < 0 || n_a < 0 || n_vs + n_bs + n_a < 1) return MINF_ERR_INVALID_ARG;
+  if (n_vs > 0) {
+    if (!vs_heads || add_seg(p, POL_VS, vs_heads, n_vs) != MINF_OK || !vs_index_ok(vs_idx))
+      return MINF_ERR_INVALID_ARG;
+    if (k_v < 1 || k_s < 1 || k_v > s->N || k_s > s->N) return MINF_ERR_INVALID_ARG;
+    set_vs_index(p, s, vs_idx, k_v, k_s);
+  }
+  if (n_bs > 0) {
+    if (!bs_heads || add_seg(p, POL_BS, bs_heads, n_bs) != MINF_OK || !blk_idx || !blk_cnt || k_b < 1)
+      return MINF_ERR_INVALID_ARG;
+    p.blk_idx = blk_idx;
+    p.blk_cnt = blk_cnt;
+    p.k_b = k_b;
+  }
+  if (n_a > 0) {
+    if (!a_heads || add_seg(p, POL_ASHAPE, a_heads, n_a) != MINF_OK || n_sink < 0 || n_local < 1)
+      return MINF_ERR_INVALID_ARG;
+    p.n_sink = n_sink;
+    p.n_local = n_local;
+  }
+  return attn_launch(s, p, stream);
 }
 
 minf_status minf_get_device_status(void* ws, void* stream) {

@@ -1,5 +1,13 @@
-// Causal (sparse) attention mainloop for sm_100a: one CTA per (batch, head,
-// 128-row query tile), warp-specialized.
+// Causal (sparse) attention mainloop for sm_100a: one CTA per work item, a
+// (batch, head, 128-row query tile), warp-specialized.  One launch can hold
+// the heads of up to three patterns, so that a whole layer of mixed patterns
+// is one grid ("MInference 1.0" summary, "Summary": a pattern per head,
+// attention over the indices only).  The grid takes the patterns in turn and
+// within a pattern one head after the other, each head's query tiles from
+// the bottom of the causal triangle up: the CTAs resident at a time share
+// one head's K and V in L2, and the light items (a head's first tiles, and
+// the Block-Sparse and A-shape heads after the Vertical-Slash ones) fill the
+// end of the launch.
 //
 //   warps 0-3  softmax warpgroup 0: key columns 0-63 of every tile  (thread = query row)
 //   warps 4-7  softmax warpgroup 1: key columns 64-127 of every tile
@@ -401,8 +409,8 @@ struct Producer {
   }
 };
 
-template <int D, int POL>
-__device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi, int qt) {
+template <int D>
+__device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int POL, int nh, int b, int hi, int qt) {
   const int R = qt * 128;
   const int lane = P.lane;
   if (POL == POL_DENSE) {
@@ -428,7 +436,7 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi
       interval(lloc, R + 127);
     }
   } else if (POL == POL_VS) {
-    const size_t hrow = (size_t)b * p.nh + hi;
+    const size_t hrow = (size_t)b * nh + hi;
     const int* tg = p.tgrp + hrow * p.k_s * 2;
     const int G = p.tgrp_cnt[hrow];
     const uint32_t* W = p.wmap + hrow * p.wmap_words;
@@ -533,7 +541,7 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi
     // The same key ranges as the band variant at 128-row granularity (one per
     // offset group of gap 128), masked element by element by the softmax from
     // the offset and key bitmaps; then the tile's own vertical list.
-    const size_t hrow = (size_t)b * p.nh + hi;
+    const size_t hrow = (size_t)b * nh + hi;
     const int* tg = p.tgrp + hrow * p.k_s * 2;
     const int G = p.tgrp_cnt[hrow];
     int top = 0;
@@ -575,7 +583,7 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi
     }
     if (n_staged > 0 && P.ok) P.emit_gather(n_staged);
   } else if (POL == POL_BS) {
-    const size_t hrow = (size_t)b * p.nh + hi;
+    const size_t hrow = (size_t)b * nh + hi;
     const int nb = p.N / 64;
     const int b0 = R / 64, b1 = b0 + 1;
     const int* s0 = p.blk_idx + (hrow * nb + b0) * (size_t)p.k_b;
@@ -648,7 +656,7 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int b, int hi
   }
 }
 
-template <int D, int POL>
+template <int D, bool EXACT>
 __global__ void __launch_bounds__(320, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
@@ -658,11 +666,21 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int nqt = p.N / 128;
-  const int qt = nqt - 1 - blockIdx.x;  // heaviest query tiles first
-  const int hi = blockIdx.y;
-  const int b = blockIdx.z;
-  const int head = p.heads ? p.heads[hi] : hi;
+  // work item: the segment (pattern), then (batch, head), then the query
+  // tile from the heaviest down
+  int x = (int)blockIdx.x;
+  int seg = 0;
+  while (seg < p.nseg - 1 && x >= p.B * p.seg[seg].nh * p.nqt) {
+    x -= p.B * p.seg[seg].nh * p.nqt;
+    ++seg;
+  }
+  const int qt = p.nqt - 1 - x % p.nqt;
+  const int bh = x / p.nqt;
+  const int b = bh / p.seg[seg].nh;
+  const int hi = bh % p.seg[seg].nh;
+  const int pol = p.seg[seg].pol;
+  const int nh = p.seg[seg].nh;
+  const int head = p.seg[seg].heads ? __ldg(p.seg[seg].heads + hi) : hi;
   const int kvh = head / p.group;
   const int R = qt * 128;
 
@@ -758,9 +776,9 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
     // Failure-detection test hook: the first CTA withholds every key tile,
     // so its consumers' bounded waits run out and the call reports a timeout.
-    const bool withhold = p.status->withhold != 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+    const bool withhold = p.status->withhold != 0 && blockIdx.x == 0;
     if (!withhold) {
-      produce_tiles<D, POL>(P, p, b, hi, qt);
+      produce_tiles<D>(P, p, pol, nh, b, hi, qt);
       if (lane == 0 && P.ok) atomicAdd(&p.status->tiles, (unsigned long long)P.t);
       P.emit_end();
     }
@@ -860,10 +878,10 @@ __global__ void __launch_bounds__(320, 1)
       // element-exact tiles: the bitmap words of this row's window are
       // requested before waiting for the scores
       Window64 xs, xv;
-      const bool exact = POL == POL_VS_EXACT && (flags & F_EXACT);
+      const bool exact = EXACT && (flags & F_EXACT);
       const int jw = dd.j0[wg];  // RANGE tiles: first key of this warpgroup's chunk
       if (exact) {
-        const size_t hb = ((size_t)b * p.nh + hi) * p.bits_words;
+        const size_t hb = ((size_t)b * nh + hi) * p.bits_words;
         xs.load(p.sbits + hb, i - jw - 63);
         xv.load(p.vbits + hb, jw);
       }
@@ -1090,34 +1108,27 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ------------------------------------------------------------------ launch
-template <int D, int POL>
+template <int D, bool EXACT>
 static cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                const CUtensorMap& tk2, const CUtensorMap& tv2, const AttnParams& p,
                                cudaStream_t stream) {
   using C = AttnCfg<D>;
-  auto kfn = attn_kernel<D, POL>;
+  auto kfn = attn_kernel<D, EXACT>;
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.N / 128, p.nh, p.B);
-  kfn<<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, tk2, tv2, p);
+  kfn<<<p.nitems, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, tk2, tv2, p);
   return cudaGetLastError();
 }
 
-cudaError_t attn_dispatch(int d, int pol, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+cudaError_t attn_dispatch(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tk2, const CUtensorMap& tv2, const AttnParams& p, cudaStream_t stream) {
-#define MINF_CASE(DD, PP) \
-  if (d == DD && pol == PP) return launch_attn<DD, PP>(tq, tk, tv, tk2, tv2, p, stream);
-  MINF_CASE(64, POL_DENSE)
-  MINF_CASE(64, POL_ASHAPE)
-  MINF_CASE(64, POL_VS)
-  MINF_CASE(64, POL_BS)
-  MINF_CASE(128, POL_DENSE)
-  MINF_CASE(128, POL_ASHAPE)
-  MINF_CASE(128, POL_VS)
-  MINF_CASE(128, POL_BS)
-  MINF_CASE(64, POL_VS_EXACT)
-  MINF_CASE(128, POL_VS_EXACT)
-#undef MINF_CASE
+  // the element-exact reading has a kernel of its own (its bitmap windows
+  // need registers in the softmax); it is never mixed with other patterns
+  const bool exact = p.nseg == 1 && p.seg[0].pol == POL_VS_EXACT;
+  if (d == 64) return exact ? launch_attn<64, true>(tq, tk, tv, tk2, tv2, p, stream)
+                            : launch_attn<64, false>(tq, tk, tv, tk2, tv2, p, stream);
+  if (d == 128) return exact ? launch_attn<128, true>(tq, tk, tv, tk2, tv2, p, stream)
+                             : launch_attn<128, false>(tq, tk, tv, tk2, tv2, p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -16,26 +16,37 @@ struct DevStatus;
 
 enum { POL_DENSE = 0, POL_ASHAPE = 1, POL_VS = 2, POL_BS = 3, POL_VS_EXACT = 4 };
 
+// One pattern's heads in an attention launch.  Work items are 128-row query
+// tiles of one (batch, head); a launch may hold up to three segments (one per
+// pattern), whose items interleave.
+struct AttnSeg {
+  int pol;
+  const int32_t* heads;  // nh query-head ids, or NULL for heads 0 .. nh-1
+  int nh;
+};
+
 struct AttnParams {
   const __nv_bfloat16* Q;
   const __nv_bfloat16* K;
   const __nv_bfloat16* V;
   __nv_bfloat16* O;
   float* lse;
-  const int32_t* heads;
-  int nh;
+  AttnSeg seg[3];
+  int nseg, nh_total;
+  int nqt, nitems;      // query tiles N / 128; items = nqt * B * nh_total
   int B, Hq, Hkv, N, group;
   float scale_log2;  // softmax scale * log2(e)
   // A-shape
   int n_sink, n_local;
-  // Vertical-Slash index
+  // Vertical-Slash index (band reading: tgrp, wmap, per-64-row-block vcnt /
+  // vidx; exact reading: tgrp, twmap, sbits, vbits, per-128-row-tile lists)
   const int32_t* tgrp;
   const int32_t* tgrp_cnt;
   const uint32_t* wmap;
+  const uint32_t* twmap;
   const int32_t* vcnt;
   const int32_t* vidx;
-  int k_s, k_v, wmap_words;
-  // element-exact Vertical-Slash (vcnt / vidx then hold per-128-row-tile lists)
+  int k_s, k_v, wmap_words, twmap_words;
   const uint32_t* sbits;
   const uint32_t* vbits;
   int bits_words;
@@ -47,8 +58,9 @@ struct AttnParams {
 };
 
 // tq: Q with 128-row boxes; tk/tv: K and V with 64-row boxes; tk2/tv2: K and V
-// with 128-row boxes (all 128-byte swizzled, 64 columns wide)
-cudaError_t attn_dispatch(int d, int pol, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+// with 128-row boxes (all 128-byte swizzled, 64 columns wide).  One CTA per
+// work item.
+cudaError_t attn_dispatch(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tk2, const CUtensorMap& tv2, const AttnParams& p, cudaStream_t stream);
 
 // ---- estimation / index kernels (estimate.cu, index.cu)

@@ -31,6 +31,27 @@ class LayerPlan:
         return minf.Shape(w.B, w.Hq, w.Hkv, w.N, w.d, 0.0)
 
 
+def kv_group_slice(w: Workload, rank: int, world: int):
+    """The share of rank ``rank`` when one layer is split across ``world``
+    GPUs by KV-head group: KV heads [hk0, hk1) and their query heads
+    [hq0, hq1) (contiguous, since query head h reads KV head h // g).  Heads
+    are independent, so the shares need no exchange; O stays head-sharded."""
+    if world < 1 or w.Hkv % world:
+        raise ValueError(f"{w.Hkv} KV heads do not split over {world} ranks")
+    per = w.Hkv // world
+    hk0, hk1 = rank * per, (rank + 1) * per
+    return hk0 * w.group, hk1 * w.group, hk0, hk1
+
+
+def local_workload(w: Workload, rank: int, world: int) -> Workload:
+    """The workload one rank runs under :func:`kv_group_slice`: its query and
+    KV heads only, with their rows of the head -> pattern table."""
+    import dataclasses
+    hq0, hq1, hk0, hk1 = kv_group_slice(w, rank, world)
+    return dataclasses.replace(w, name=f"{w.name}_kv{hk0}-{hk1 - 1}", Hq=hq1 - hq0, Hkv=hk1 - hk0,
+                               patterns=list(w.patterns[hq0:hq1]))
+
+
 def make_plan(w: Workload, device="cuda") -> LayerPlan:
     dev = torch.device(device)
     plan = LayerPlan(w, dev)
@@ -59,6 +80,7 @@ def make_plan(w: Workload, device="cuda") -> LayerPlan:
     if ah:
         plan.a_heads = torch.tensor(ah, **i32)
         plan.bufs["ws_a"] = minf.workspace(minf.OP_ATTN_ASHAPE, shp, len(ah), device=dev)
+    plan.bufs["ws_attn"] = minf.workspace(minf.OP_SPARSE_ATTN_LAYER, shp, len(vs) + len(bs) + len(ah), device=dev)
     return plan
 
 
@@ -66,24 +88,29 @@ def make_plan(w: Workload, device="cuda") -> LayerPlan:
 TOPK_LONG_ROW = 32768
 
 
-def launches_per_step(plan: LayerPlan) -> int:
+def launches_per_step(plan: LayerPlan, fused: bool = True) -> int:
     """Kernels one run_layer call launches: VS estimation (two score passes,
     row combine, slash combine, two top-k), VS index build 3, BS estimation
-    3 (pool, pooled scores, top-k), and one attention launch per pattern."""
+    3 (pool, pooled scores, top-k), and the attention: one launch for every
+    head (fused) or one per pattern."""
     n = 0
     if plan.vs_heads is not None:
         topk = 9 if plan.w.N > TOPK_LONG_ROW else 1
-        n += 4 + 2 * topk + 3 + 1
+        n += 4 + 2 * topk + 3
     if plan.bs_heads is not None:
-        n += 3 + 1
-    if plan.a_heads is not None:
+        n += 3
+    if fused:
         n += 1
+    else:
+        n += sum(1 for h in (plan.vs_heads, plan.bs_heads, plan.a_heads) if h is not None)
     return n
 
 
-def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None, marks=None):
+def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None, marks=None, fused: bool = True):
     """Estimation, index build and sparse attention for every head of the
-    layer, in stream order; O (and LSE) are filled head by head.  ``marks``
+    layer, in stream order; O (and LSE) are filled head by head.  With
+    ``fused`` the attention of all heads runs as one launch
+    (minf_sparse_attn_layer), otherwise as one launch per pattern.  ``marks``
     (optional) gets ``mark(name)`` calls, ``<phase>:pre`` and ``<phase>:post``,
     around every call of the layer."""
     mark = marks.mark if marks is not None else (lambda name: None)
@@ -92,38 +119,50 @@ def run_layer(plan: LayerPlan, q, k, v, o, lse=None, stream=None, marks=None):
     L = minf.lib()
     st = minf._stream(stream)
     P = minf._p
-    if plan.vs_heads is not None:
-        nv = plan.vs_heads.numel()
+    nv = plan.vs_heads.numel() if plan.vs_heads is not None else 0
+    nbh = plan.bs_heads.numel() if plan.bs_heads is not None else 0
+    na = plan.a_heads.numel() if plan.a_heads is not None else 0
+    ic = b["vs_index"].c() if nv else None
+    if nv:
         mark("vs_est:pre")
         minf._check("minf_estimate_vs", L.minf_estimate_vs(
             minf.ctypes.byref(shp), P(q), P(k), P(plan.vs_heads), nv, w.last_q, w.k_v, w.k_s,
             P(b["v_idx"]), P(b["s_idx"]), None, None, P(b["ws_vs_est"]), b["ws_vs_est"].numel(), st))
         mark("vs_est:post")
-        ic = b["vs_index"].c()
         mark("vs_index:pre")
         minf._check("minf_build_index", L.minf_build_index(
             minf.ctypes.byref(shp), nv, P(b["v_idx"]), w.k_v, P(b["s_idx"]), w.k_s, minf.ctypes.byref(ic),
             P(b["ws_vs_idx"]), b["ws_vs_idx"].numel(), st))
         mark("vs_index:post")
-        mark("vs_attn:pre")
-        minf._check("minf_sparse_attn_vs", L.minf_sparse_attn_vs(
-            minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.vs_heads), nv, minf.ctypes.byref(ic),
-            w.k_v, w.k_s, P(o), P(lse), P(b["ws_vs_attn"]), b["ws_vs_attn"].numel(), st))
-        mark("vs_attn:post")
-    if plan.bs_heads is not None:
-        nbh = plan.bs_heads.numel()
+    if nbh:
         mark("bs_est:pre")
         minf._check("minf_estimate_bs", L.minf_estimate_bs(
             minf.ctypes.byref(shp), P(q), P(k), P(plan.bs_heads), nbh, w.block, w.k_b,
             P(b["blk_idx"]), P(b["blk_cnt"]), None, P(b["ws_bs_est"]), b["ws_bs_est"].numel(), st))
         mark("bs_est:post")
+    if fused:
+        mark("attn:pre")
+        minf._check("minf_sparse_attn_layer", L.minf_sparse_attn_layer(
+            minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.vs_heads) if nv else None, nv,
+            minf.ctypes.byref(ic) if nv else None, w.k_v, w.k_s,
+            P(plan.bs_heads) if nbh else None, nbh, P(b["blk_idx"]) if nbh else None,
+            P(b["blk_cnt"]) if nbh else None, w.k_b, P(plan.a_heads) if na else None, na,
+            w.n_sink, w.n_local, P(o), P(lse), P(b["ws_attn"]), b["ws_attn"].numel(), st))
+        mark("attn:post")
+        return o, lse
+    if nv:
+        mark("vs_attn:pre")
+        minf._check("minf_sparse_attn_vs", L.minf_sparse_attn_vs(
+            minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.vs_heads), nv, minf.ctypes.byref(ic),
+            w.k_v, w.k_s, P(o), P(lse), P(b["ws_vs_attn"]), b["ws_vs_attn"].numel(), st))
+        mark("vs_attn:post")
+    if nbh:
         mark("bs_attn:pre")
         minf._check("minf_sparse_attn_bs", L.minf_sparse_attn_bs(
             minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.bs_heads), nbh, P(b["blk_idx"]),
             P(b["blk_cnt"]), w.k_b, P(o), P(lse), P(b["ws_bs_attn"]), b["ws_bs_attn"].numel(), st))
         mark("bs_attn:post")
-    if plan.a_heads is not None:
-        na = plan.a_heads.numel()
+    if na:
         mark("a_attn:pre")
         minf._check("minf_attn_ashape", L.minf_attn_ashape(
             minf.ctypes.byref(shp), P(q), P(k), P(v), P(plan.a_heads), na, w.n_sink, w.n_local,

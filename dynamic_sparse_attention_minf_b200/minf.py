@@ -19,12 +19,13 @@ OK = 0
 STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error",
                 4: "workspace too small", 5: "device timeout", 6: "device bounds"}
 OP_ESTIMATE_VS, OP_ESTIMATE_BS, OP_BUILD_INDEX, OP_SPARSE_ATTN_VS, OP_SPARSE_ATTN_BS, \
-    OP_ATTN_ASHAPE, OP_DENSE_ATTN, OP_BUILD_INDEX_EXACT, OP_SPARSE_ATTN_VS_EXACT = range(9)
+    OP_ATTN_ASHAPE, OP_DENSE_ATTN, OP_BUILD_INDEX_EXACT, OP_SPARSE_ATTN_VS_EXACT, OP_SPARSE_ATTN_LAYER = range(10)
 
 EXPORTS = ["minf_vs_wmap_words", "minf_workspace_size", "minf_estimate_vs", "minf_estimate_bs",
            "minf_build_index", "minf_sparse_attn_vs", "minf_sparse_attn_bs", "minf_attn_ashape",
            "minf_dense_attn", "minf_get_device_status", "minf_status_string", "minf_vs_bits_words",
-           "minf_vs_twmap_words", "minf_build_index_exact", "minf_sparse_attn_vs_exact"]
+           "minf_vs_twmap_words", "minf_build_index_exact", "minf_sparse_attn_vs_exact",
+           "minf_sparse_attn_layer"]
 
 
 class MinfError(RuntimeError):
@@ -80,12 +81,14 @@ def lib():
         L.minf_sparse_attn_bs.argtypes = [sp, vp, vp, vp, vp, i, vp, vp, i, vp, vp, vp, sz, vp]
         L.minf_attn_ashape.argtypes = [sp, vp, vp, vp, vp, i, i, i, vp, vp, vp, sz, vp]
         L.minf_dense_attn.argtypes = [sp, vp, vp, vp, vp, i, vp, vp, vp, sz, vp]
+        L.minf_sparse_attn_layer.argtypes = [sp, vp, vp, vp, vp, i, ctypes.POINTER(_VsIndexC), i, i, vp, i, vp,
+                                             vp, i, vp, i, i, i, vp, vp, vp, sz, vp]
         L.minf_get_device_status.argtypes = [vp, vp]
         L.minf_status_string.argtypes = [st]
         L.minf_status_string.restype = ctypes.c_char_p
         for fn in ("minf_estimate_vs", "minf_estimate_bs", "minf_build_index", "minf_sparse_attn_vs",
                    "minf_sparse_attn_bs", "minf_attn_ashape", "minf_dense_attn", "minf_get_device_status",
-                   "minf_build_index_exact", "minf_sparse_attn_vs_exact"):
+                   "minf_build_index_exact", "minf_sparse_attn_vs_exact", "minf_sparse_attn_layer"):
             getattr(L, fn).restype = st
         _lib = L
     return _lib
@@ -324,6 +327,28 @@ def minf_dense_attn(q, k, v, heads=None, o=None, lse=None, want_lse=True, scale=
     _check("minf_dense_attn", lib().minf_dense_attn(
         ctypes.byref(shp), _p(q), _p(k), _p(v), _p(hd), nh, _p(o), _p(lse), _p(ws), ws.numel(),
         _stream(stream)))
+    return o, lse
+
+
+def minf_sparse_attn_layer(q, k, v, vs_heads=None, vs_index: VSIndex | None = None, bs_heads=None,
+                           blk_idx=None, blk_cnt=None, a_heads=None, n_sink=0, n_local=1, o=None, lse=None,
+                           want_lse=True, scale=0.0, ws=None, stream=None):
+    """Every head of a mixed-pattern layer in one launch (see
+    minf_sparse_attn_layer in include/minf.h); a group whose heads are None or
+    empty is left out."""
+    shp = shape_of(q, k, scale)
+    vh, bh, ah = (_heads(h, q.device) for h in (vs_heads, bs_heads, a_heads))
+    nv, nb, na = (0 if h is None else h.numel() for h in (vh, bh, ah))
+    o, lse = _out(q, o, lse, want_lse)
+    if ws is None:
+        ws = workspace(OP_SPARSE_ATTN_LAYER, shp, max(1, nv + nb + na), device=q.device)
+    ic = vs_index.c() if (nv and vs_index is not None) else None
+    _check("minf_sparse_attn_layer", lib().minf_sparse_attn_layer(
+        ctypes.byref(shp), _p(q), _p(k), _p(v), _p(vh) if nv else None, nv,
+        ctypes.byref(ic) if ic is not None else None, vs_index.k_v if nv else 0, vs_index.k_s if nv else 0,
+        _p(bh) if nb else None, nb, _p(blk_idx) if nb else None, _p(blk_cnt) if nb else None,
+        blk_idx.shape[-1] if nb else 0, _p(ah) if na else None, na, n_sink, n_local, _p(o), _p(lse),
+        _p(ws), ws.numel(), _stream(stream)))
     return o, lse
 
 

@@ -288,6 +288,33 @@ minf_status minf_sparse_attn_vs_exact(const minf_shape* shape, const minf_bf16* 
                                       const minf_vs_exact_index* idx, int k_v, int k_s, minf_bf16* O,
                                       float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * One launch for a whole layer of mixed patterns.
+ * ------------------------------------------------------------------------- */
+enum { MINF_OP_SPARSE_ATTN_LAYER = 9 };
+
+/*
+ * Attention of every head of a layer whose heads follow different patterns
+ * (summary page, "Summary": a pattern per head, chosen offline; attention over
+ * the estimated indices only), in one persistent launch: the Vertical-Slash
+ * heads vs_heads[n_vs] with the index vs_idx (as minf_sparse_attn_vs), the
+ * Block-Sparse heads bs_heads[n_bs] with blk_idx / blk_cnt (as
+ * minf_sparse_attn_bs) and the A-shape heads a_heads[n_a] (as
+ * minf_attn_ashape).  Per-head index arrays are laid out [B, n, ...] in the
+ * order of their own head list.  Any of the three groups may be empty (n = 0,
+ * pointers ignored); the head lists must be disjoint and hold at most Hq
+ * heads together.  The results equal those of the three separate calls; the
+ * work items of all heads are interleaved heaviest first, so the light
+ * Block-Sparse and A-shape heads fill the end of the launch instead of
+ * running launches of their own.  lse may be NULL.
+ */
+minf_status minf_sparse_attn_layer(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K,
+                                   const minf_bf16* V, const int32_t* vs_heads, int n_vs,
+                                   const minf_vs_index* vs_idx, int k_v, int k_s, const int32_t* bs_heads,
+                                   int n_bs, const int32_t* blk_idx, const int32_t* blk_cnt, int k_b,
+                                   const int32_t* a_heads, int n_a, int n_sink, int n_local, minf_bf16* O,
+                                   float* lse, void* ws, size_t ws_bytes, void* stream);
+
 /*
  * Synchronizes `stream`, returns the device status word of `ws` (MINF_OK when
  * no kernel reported an error since the last call) and clears it.

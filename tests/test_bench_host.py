@@ -18,21 +18,28 @@ def _plan(cid):
 
 
 def test_launches_per_step_matches_launch_list_profile():
-    """The count the bench reports equals the kernels ncu listed per layer."""
+    """The count the bench reports equals the kernels ncu listed per layer:
+    the run holds layers with one attention launch for every head (the
+    product path) and layers with one attention launch per pattern."""
     n = layer.launches_per_step(_plan(4))
+    n_sep = layer.launches_per_step(_plan(4), fused=False)
     text = open(os.path.join(bench.ROOT, "profiles", "launches_llama3_8b_layer_n1m.md")).read()
-    per_layer = int(re.search(r"(\d+) launches per layer", text).group(1))
-    layers = 9
+    m = re.search(r"(\d+) launches of libminf kernels in all = (\d+) x (\d+) \+ (\d+) x (\d+)", text)
+    total, lf, nf, ls, ns = (int(g) for g in m.groups())
     listed = sum(int(c) for c in re.findall(r"^\| `minf::[^|]*\| (\d+) \|", text, re.M))
-    assert n == per_layer == listed // layers
-    assert listed % layers == 0
+    assert (nf, ns) == (n, n_sep) == (29, 31)
+    assert listed == total == lf * nf + ls * ns
+    attn = sum(int(c) for c in re.findall(r"^\| `minf::attn_kernel[^|]*\| (\d+) \|", text, re.M))
+    assert attn == lf + 3 * ls
 
 
 def test_launches_per_step_other_layers():
     # 512K, Vertical-Slash heads only: estimation 4 + two 9-launch top-k, index 3, attention 1
     assert layer.launches_per_step(_plan(3)) == 26
-    # 128K mixed layer: the same kernels as the 1M layer
-    assert layer.launches_per_step(_plan(2)) == 31
+    # 128K mixed layer: the same kernels as the 1M layer (one attention launch for all heads)
+    assert layer.launches_per_step(_plan(2)) == 29
+    # one attention launch per pattern instead
+    assert layer.launches_per_step(_plan(2), fused=False) == 31
 
 
 def test_digest_ignores_comments_and_whitespace():

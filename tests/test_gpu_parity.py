@@ -105,8 +105,10 @@ def _vs_pipeline(w, heads, rows=None):
     return gv, gs
 
 
-def test_vs_pipeline_small():
-    w = wl.small(Hq=4, Hkv=2, N=2048, d=128, seed=21, k_v=64, k_s=128)
+@pytest.mark.parametrize("N", [2048, 1152])
+def test_vs_pipeline_small(N):
+    """N = 1152 is nine 128-row tiles: the last pair of query tiles has one tile."""
+    w = wl.small(Hq=4, Hkv=2, N=N, d=128, seed=21, k_v=64, k_s=128)
     _vs_pipeline(w, [0, 3])
 
 
@@ -176,8 +178,9 @@ def _bs_pipeline(w, heads, rows=None):
     return flips
 
 
-def test_bs_pipeline_small():
-    w = wl.small(Hq=4, Hkv=2, N=2048, d=128, seed=4, bias="block", patterns=[wl.PAT_BS] * 4, k_b=7)
+@pytest.mark.parametrize("N,d", [(2048, 128), (640, 128), (1152, 64)])
+def test_bs_pipeline_small(N, d):
+    w = wl.small(Hq=4, Hkv=2, N=N, d=d, seed=4, bias="block", patterns=[wl.PAT_BS] * 4, k_b=7)
     _bs_pipeline(w, [1, 2])
 
 
@@ -283,9 +286,10 @@ def _vs_exact_check(w, heads, V_sets, S_sets, q, k, v, qn, kn, vn):
     return o, lse
 
 
-def test_vs_exact_pipeline_small():
+@pytest.mark.parametrize("N", [2048, 896])
+def test_vs_exact_pipeline_small(N):
     """Estimated V and S (GPU top-k, checked against the oracle), then the exact variant."""
-    w = wl.small(Hq=4, Hkv=2, N=2048, d=128, seed=41, k_v=64, k_s=128)
+    w = wl.small(Hq=4, Hkv=2, N=N, d=128, seed=41, k_v=64, k_s=128)
     q, k, v, qn, kn, vn = _inputs(w)
     sc = orc.default_scale(w.d)
     heads = [1, 2]
