@@ -69,17 +69,18 @@ struct AttnCfg {
   static constexpr int kRegion = 128 * 128;                 // bytes: 128 rows x 128 B
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = 128 * D * 2;
-  static constexpr int kStages = (D == 128) ? 3 : 4;
+  static constexpr int kKStages = (D == 128) ? 3 : 4;  // K slots (with their descriptors)
+  static constexpr int kVStages = (D == 128) ? 3 : 4;  // V slots
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kStages * kKVBytes;
-  static constexpr int kOffDesc = kOffV + kStages * kKVBytes;
-  static constexpr int kOffSCols = kOffDesc + kStages * (int)sizeof(TileDesc);
+  static constexpr int kOffV = kOffK + kKStages * kKVBytes;
+  static constexpr int kOffDesc = kOffV + kVStages * kKVBytes;
+  static constexpr int kOffSCols = kOffDesc + kKStages * (int)sizeof(TileDesc);
   static constexpr int kOffSBits = kOffSCols + 160 * 4;
   static constexpr int kOffBars = kOffSBits + 160;
-  // barriers: k_full[S], v_full[S], k_empty[S], v_empty[S], d_empty[S], s_full[2], p_full[2],
-  // q_full, mma_done
-  static constexpr int kNumBars = 5 * kStages + 6;
+  // barriers: k_full, k_empty, d_empty [kKStages]; v_full, v_empty [kVStages];
+  // s_full[2], p_full[2], q_full, mma_done
+  static constexpr int kNumBars = 3 * kKStages + 2 * kVStages + 6;
   static constexpr int kOffMisc = kOffBars + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16;
   static_assert(kSmem <= 232448, "shared memory budget");
@@ -177,31 +178,31 @@ struct Producer {
   int t;        // tiles whose K side (and descriptor) has been emitted
   int tv;       // tiles whose V side has been emitted: t - 1 (a range tile's V lags) or t
   int vj0[2];   // key chunks of tile tv while its V lags
-  int pending;  // stage whose gathered copies are issued but not yet signalled
+  int pend_k, pend_v;  // K and V slots of the gathered tile whose copies are issued but not yet signalled
   volatile int* abort;
   DevStatus* st;
   bool ok;
 
   __device__ void flush_pending() {
-    if (pending >= 0) {
+    if (pend_k >= 0) {
       cp_async_wait<0>();
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&k_full[pending]);
-        mbar_arrive(&v_full[pending]);
+        mbar_arrive(&k_full[pend_k]);
+        mbar_arrive(&v_full[pend_v]);
       }
-      pending = -1;
+      pend_k = pend_v = -1;
     }
   }
 
   // Claims the K slot and the descriptor of tile t: S = Q K^T of tile t - S
   // is done and the softmax warps have read its descriptor.  False on abort.
   __device__ bool acquire_k(int& stage) {
-    stage = t % C::kStages;
-    if (t >= C::kStages) {
+    stage = t % C::kKStages;
+    if (t >= C::kKStages) {
       flush_pending();
-      const uint32_t par = ((t / C::kStages) - 1) & 1;
+      const uint32_t par = ((t / C::kKStages) - 1) & 1;
       if (!warp_wait(&k_empty[stage], par, abort, st, 1) || !warp_wait(&d_empty[stage], par, abort, st, 14)) {
         ok = false;
         return false;
@@ -212,10 +213,10 @@ struct Producer {
 
   // Claims the V slot of tile u: P V of tile u - S is done.
   __device__ bool acquire_v(int u, int& stage) {
-    stage = u % C::kStages;
-    if (u >= C::kStages) {
+    stage = u % C::kVStages;
+    if (u >= C::kVStages) {
       flush_pending();
-      if (!warp_wait(&v_empty[stage], ((u / C::kStages) - 1) & 1, abort, st, 15)) {
+      if (!warp_wait(&v_empty[stage], ((u / C::kVStages) - 1) & 1, abort, st, 15)) {
         ok = false;
         return false;
       }
@@ -329,16 +330,17 @@ struct Producer {
     }
     cp_async_commit();
     // signal the previous gathered tile, keep this one in flight
-    if (pending >= 0) {
+    if (pend_k >= 0) {
       cp_async_wait<1>();
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&k_full[pending]);
-        mbar_arrive(&v_full[pending]);
+        mbar_arrive(&k_full[pend_k]);
+        mbar_arrive(&v_full[pend_v]);
       }
     }
-    pending = stage;  // K and V slots of a tile have the same index
+    pend_k = stage;
+    pend_v = vstage;
     ++t;
     ++tv;
   }
@@ -391,7 +393,7 @@ struct Producer {
 
   // Waits (bounded, ignoring the abort flag) until every copy this producer
   // started has landed, so that the CTA never exits with copies in flight:
-  // the last kStages tiles of each ring (older ones were waited for when
+  // the last tiles of each ring (older ones were waited for when
   // their slots were reused).  The slots carry no per-stage bookkeeping
   // (an array indexed by stage would move the producer's state to local
   // memory).
@@ -400,10 +402,10 @@ struct Producer {
     __syncwarp();
     if (lane == 0) {
       int dummy = 0;
-      for (int u = max(0, t - C::kStages); u < t; ++u)
-        mbar_wait(&k_full[u % C::kStages], (u / C::kStages) & 1, &dummy, st, 9);
-      for (int u = max(0, tv - C::kStages); u < tv; ++u)
-        mbar_wait(&v_full[u % C::kStages], (u / C::kStages) & 1, &dummy, st, 9);
+      for (int u = max(0, t - C::kKStages); u < t; ++u)
+        mbar_wait(&k_full[u % C::kKStages], (u / C::kKStages) & 1, &dummy, st, 9);
+      for (int u = max(0, tv - C::kVStages); u < tv; ++u)
+        mbar_wait(&v_full[u % C::kVStages], (u / C::kVStages) & 1, &dummy, st, 9);
     }
     __syncwarp();
   }
@@ -687,11 +689,11 @@ __global__ void __launch_bounds__(320, 1)
   TileDesc* desc = reinterpret_cast<TileDesc*>(smem + C::kOffDesc);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
   uint64_t* k_full = bars;
-  uint64_t* v_full = bars + C::kStages;
-  uint64_t* k_empty = bars + 2 * C::kStages;  // S = Q K^T of the slot's tile is done
-  uint64_t* v_empty = bars + 3 * C::kStages;  // P V of the slot's tile is done
-  uint64_t* d_empty = bars + 4 * C::kStages;  // the softmax warps have read the descriptor
-  uint64_t* s_full = bars + 5 * C::kStages;
+  uint64_t* k_empty = bars + C::kKStages;      // S = Q K^T of the slot's tile is done
+  uint64_t* d_empty = bars + 2 * C::kKStages;  // the softmax warps have read the descriptor
+  uint64_t* v_full = bars + 3 * C::kKStages;
+  uint64_t* v_empty = v_full + C::kVStages;    // P V of the slot's tile is done
+  uint64_t* s_full = v_empty + C::kVStages;
   uint64_t* p_full = s_full + 2;
   uint64_t* q_full = p_full + 2;
   uint64_t* mma_done = q_full + 1;
@@ -708,12 +710,14 @@ __global__ void __launch_bounds__(320, 1)
   }
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < C::kKStages; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
       mbar_init(&k_empty[s], 1);
-      mbar_init(&v_empty[s], 1);
       mbar_init(&d_empty[s], 256);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&s_full[w], 1);
@@ -758,7 +762,7 @@ __global__ void __launch_bounds__(320, 1)
     P.t = 0;
     P.tv = 0;
     P.vj0[0] = P.vj0[1] = 0;
-    P.pending = -1;
+    P.pend_k = P.pend_v = -1;
     P.abort = abort;
     P.st = p.status;
     P.ok = true;
@@ -797,9 +801,9 @@ __global__ void __launch_bounds__(320, 1)
     // warpgroup w's bf16 P occupies TMEM columns 64w .. 64w+31 of the buffer
     auto issue_pv = [&](int tp) -> bool {
       const int bp = tp & 1;
-      const int sp = tp % C::kStages;
+      const int sp = tp % C::kVStages;
       if (!warp_wait(&p_full[bp], (tp >> 1) & 1, abort, p.status, 3)) return false;
-      if (!warp_wait(&v_full[sp], (tp / C::kStages) & 1, abort, p.status, 4)) return false;
+      if (!warp_wait(&v_full[sp], (tp / C::kVStages) & 1, abort, p.status, 4)) return false;
       tc_fence_after();
       // descriptors of the K-steps: the stage's base plus a constant (the
       // start-address field holds address / 16 and never carries out)
@@ -822,8 +826,8 @@ __global__ void __launch_bounds__(320, 1)
     const uint64_t qd0 = sdesc_sw128(qaddr, 16, 1024);
     int t = 0, pend = -1;
     while (ok) {
-      const int st = t % C::kStages;
-      if (!warp_wait(&k_full[st], (t / C::kStages) & 1, abort, p.status, 5)) { ok = false; break; }
+      const int st = t % C::kKStages;
+      if (!warp_wait(&k_full[st], (t / C::kKStages) & 1, abort, p.status, 5)) { ok = false; break; }
       if (__all_sync(0xFFFFFFFFu, desc[st].kind == KIND_END)) break;
       // Q and K were written by TMA or by cp.async plus the producer's proxy
       // fence; the barrier alone orders them before the MMA (no tcgen05
@@ -865,8 +869,8 @@ __global__ void __launch_bounds__(320, 1)
     int n = 0;
     unsigned nnz = 0;
     for (int t = 0;; ++t) {
-      const int st = t % C::kStages;
-      if (!warp_wait(&k_full[st], (t / C::kStages) & 1, abort, p.status, 10)) break;
+      const int st = t % C::kKStages;
+      if (!warp_wait(&k_full[st], (t / C::kKStages) & 1, abort, p.status, 10)) break;
       const TileDesc& dd = desc[st];
       // kind and flags, rebuilt through one vote so that every test on them
       // is warp-uniform for the compiler too (bit l of the word is lane l's)
@@ -1023,7 +1027,7 @@ __global__ void __launch_bounds__(320, 1)
       // done after the P stores so that the scores are no longer live
       if (__any_sync(0xFFFFFFFFu, resc && n > 0)) {
         // P V of the previous tile must be complete before O is rescaled
-        if (!warp_wait(&v_empty[(n - 1) % C::kStages], ((n - 1) / C::kStages) & 1, abort, p.status, 12)) break;
+        if (!warp_wait(&v_empty[(n - 1) % C::kVStages], ((n - 1) / C::kVStages) & 1, abort, p.status, 12)) break;
         tc_fence_after();
         const uint32_t orow = srow + (wg ? C::kColO1 : C::kColO0);
 #pragma unroll 1
@@ -1050,7 +1054,7 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) atomicAdd(&p.status->nnz, c);
     }
     bool ok = !*abort;
-    if (ok && n > 0) ok = warp_wait(&v_empty[(n - 1) % C::kStages], ((n - 1) / C::kStages) & 1, abort, p.status, 13);
+    if (ok && n > 0) ok = warp_wait(&v_empty[(n - 1) % C::kVStages], ((n - 1) / C::kVStages) & 1, abort, p.status, 13);
     named_bar_sync(1, 256);
     float* xch = reinterpret_cast<float*>(smem + C::kOffK);  // all S MMAs are done: K stage 0 is free
     xch[(wg * 128 + r) * 4 + 0] = m_run;

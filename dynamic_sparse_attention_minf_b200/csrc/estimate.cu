@@ -158,7 +158,9 @@ __device__ __forceinline__ void topk_rows_body(const TopkRows& t) {
   const int forced = (t.forced_mode == 0) ? -1 : (t.forced_mode == 1) ? 0 : (row % t.rows_per_group);
   const float* sc = t.scores + (long long)row * t.row_stride;
   const int k = min(t.k, len);
-  __shared__ unsigned hist[kTopkThreads / 32][256];  // one histogram per warp
+  // long rows: one 256-bin histogram per warp (1024 threads); short rows: one
+  // 2048-bin histogram (8 KB), so that more rows' CTAs fit on an SM
+  __shared__ unsigned hist[SHORT ? 8 : kTopkThreads / 32][256];
   __shared__ unsigned long long wsum[32];
   __shared__ uint32_t sh_sel, sh_rem;
   __shared__ uint32_t ck[kTopkCap];
@@ -395,7 +397,7 @@ __device__ __forceinline__ void topk_rows_body(const TopkRows& t) {
 // One CTA per row: 1024 threads for rows too long for the short-row path
 // (only when no scratch is given), 256 for the rest.
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_rows_kernel(const TopkRows t) { topk_rows_body<false>(t); }
-__global__ void __launch_bounds__(256) topk_short_rows_kernel(const TopkRows t) { topk_rows_body<true>(t); }
+__global__ void __launch_bounds__(256, 4) topk_short_rows_kernel(const TopkRows t) { topk_rows_body<true>(t); }
 
 // ---------------------------------------------- top-k of long rows, many CTAs
 // The same selection as topk_rows_kernel, for rows too long for one CTA: the

@@ -25,7 +25,7 @@ EXPORTS = ["minf_vs_wmap_words", "minf_workspace_size", "minf_estimate_vs", "min
            "minf_build_index", "minf_sparse_attn_vs", "minf_sparse_attn_bs", "minf_attn_ashape",
            "minf_dense_attn", "minf_get_device_status", "minf_status_string", "minf_vs_bits_words",
            "minf_vs_twmap_words", "minf_build_index_exact", "minf_sparse_attn_vs_exact",
-           "minf_sparse_attn_layer"]
+           "minf_sparse_attn_layer", "minf_selftest_exp2"]
 
 
 class MinfError(RuntimeError):
@@ -81,6 +81,7 @@ def lib():
         L.minf_sparse_attn_bs.argtypes = [sp, vp, vp, vp, vp, i, vp, vp, i, vp, vp, vp, sz, vp]
         L.minf_attn_ashape.argtypes = [sp, vp, vp, vp, vp, i, i, i, vp, vp, vp, sz, vp]
         L.minf_dense_attn.argtypes = [sp, vp, vp, vp, vp, i, vp, vp, vp, sz, vp]
+        L.minf_selftest_exp2.argtypes = [vp, vp, vp, i, vp]
         L.minf_sparse_attn_layer.argtypes = [sp, vp, vp, vp, vp, i, ctypes.POINTER(_VsIndexC), i, i, vp, i, vp,
                                              vp, i, vp, i, i, i, vp, vp, vp, sz, vp]
         L.minf_get_device_status.argtypes = [vp, vp]
@@ -88,7 +89,8 @@ def lib():
         L.minf_status_string.restype = ctypes.c_char_p
         for fn in ("minf_estimate_vs", "minf_estimate_bs", "minf_build_index", "minf_sparse_attn_vs",
                    "minf_sparse_attn_bs", "minf_attn_ashape", "minf_dense_attn", "minf_get_device_status",
-                   "minf_build_index_exact", "minf_sparse_attn_vs_exact", "minf_sparse_attn_layer"):
+                   "minf_build_index_exact", "minf_sparse_attn_vs_exact", "minf_sparse_attn_layer",
+                   "minf_selftest_exp2"):
             getattr(L, fn).restype = st
         _lib = L
     return _lib
@@ -377,3 +379,11 @@ def minf_estimate_vs_noalloc(q, k, heads, k_v, k_s, last_q=64, scale=0.0, return
     _check("minf_estimate_vs_noalloc", fn(ctypes.byref(shp), _p(q), _p(k), _p(hd), nh, last_q, k_v, k_s,
                                           _p(v_idx), _p(s_idx), _p(vs), _p(ss), _stream(stream)))
     return (v_idx, s_idx, vs, ss) if return_scores else (v_idx, s_idx)
+
+
+def minf_selftest_exp2(x, stream=None):
+    """The softmax's two exponentials on device floats x: (polynomial, MUFU)."""
+    x = x.contiguous().float()
+    yp, ym = torch.empty_like(x), torch.empty_like(x)
+    _check("minf_selftest_exp2", lib().minf_selftest_exp2(_p(x), _p(yp), _p(ym), x.numel(), _stream(stream)))
+    return yp, ym

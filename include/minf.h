@@ -321,6 +321,20 @@ minf_status minf_sparse_attn_layer(const minf_shape* shape, const minf_bf16* Q, 
  */
 minf_status minf_get_device_status(void* ws, void* stream);
 
+/*
+ * Diagnostic, not part of the method: evaluates on the device the two
+ * exponentials the attention softmax uses for P = 2^(s * scale * log2 e - m),
+ * for n caller-given arguments x (device arrays of n floats each):
+ *   y_poly = the FMA-pipe routine that takes one pair of exponentials in four
+ *            (2^x = 2^round(x) * p(x - round(x)) with p the degree-3 minimax
+ *            fit of 2^f on [-1/2, 1/2] for relative error, at most 7.5e-5;
+ *            arguments below -126 are clamped to -126)
+ *   y_mufu = ex2.approx.ftz.f32 (the MUFU unit)
+ * so that a caller can check their accuracy on the GPU that runs them.
+ * Asynchronous on `stream`.
+ */
+minf_status minf_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int n, void* stream);
+
 /* Static description of a status code. */
 const char* minf_status_string(minf_status s);
 
