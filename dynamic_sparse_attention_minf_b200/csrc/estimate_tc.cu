@@ -8,7 +8,8 @@
 // quarter holds real scores: lanes 0-63 serve key columns 0-63 and lanes
 // 64-127 key columns 64-127, and all eight score warps (two per SM
 // sub-partition) work on each tile, 32 rows x 32 columns each.  The real rows
-// are the last `last_q` <= 64.  K tiles stream through a 3-stage TMA ring.
+// are the last `last_q` <= 64.  K tiles stream through a TMA ring of 2 stages
+// (pass 1, two CTAs per SM) or 3 (pass 2).
 //
 //  pass 1: each thread keeps an online (max, sum) of 2^(s * scale * log2 e)
 //          over its columns of the CTA's tiles; the four column groups of a
@@ -26,20 +27,22 @@
 
 namespace minf {
 
-template <int D>
+// Pass 1 needs no P buffer: two K stages keep its CTA under half of an SM's
+// shared memory, so that two CTAs share each SM and hide each other's waits.
+template <int D, int PASS>
 struct EstCfg {
   static constexpr int kThreads = 320;
   static constexpr int kScoreThreads = 256;
   static constexpr int kRegion = 128 * 128;
   static constexpr int kTileBytes = 128 * D * 2;  // 128 rows (Q twice) or 128 keys (K)
-  static constexpr int kStages = 3;
+  static constexpr int kStages = (PASS == 1) ? 2 : 3;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTileBytes;
   static constexpr int kOffP = kOffK + kStages * kTileBytes;  // pass 2: 2 x [64][129] fp32
   static constexpr int kPStride = 129;
   static constexpr int kPBytes = 64 * kPStride * 4;
-  static constexpr int kOffBars = kOffP + 2 * kPBytes;
-  // barriers: q_full, k_full[3], k_empty[3], s_full[2], s_free[2], mma_done
+  static constexpr int kOffBars = kOffP + (PASS == 2 ? 2 * kPBytes : 0);
+  // barriers: q_full, k_full[kStages], k_empty[kStages], s_full[2], s_free[2], mma_done
   static constexpr int kNumBars = 1 + 2 * kStages + 4 + 1;
   static constexpr int kOffMisc = kOffBars + kNumBars * 8;
   static constexpr int kOffXch = kOffMisc + 16;             // pass 1: [4][64][2] fp32
@@ -49,10 +52,10 @@ struct EstCfg {
 };
 
 template <int D, int PASS>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(320, PASS == 1 ? 2 : 1)
     vs_est_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const VsEstParams p, int tiles_per_cta, int nchunks) {
-  using C = EstCfg<D>;
+  using C = EstCfg<D, PASS>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
@@ -280,21 +283,22 @@ __global__ void __launch_bounds__(320, 1)
 template <int D>
 static cudaError_t launch_est_tc(const CUtensorMap& tq, const CUtensorMap& tk, const VsEstParams& p,
                                  cudaStream_t stream) {
-  using C = EstCfg<D>;
+  using C1 = EstCfg<D, 1>;
+  using C2 = EstCfg<D, 2>;
   const int ntiles = (p.N + 127) / 128;
   // about four CTAs per SM in all, at most 32 key tiles each
   const long long units = (long long)ntiles * p.nh * p.B;
   const int tpc = (int)std::max<long long>(1, std::min<long long>(32, (units + 591) / 592));
   const int nchunks = (ntiles + tpc - 1) / tpc;
-  cudaError_t e = cudaFuncSetAttribute(vs_est_tc_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  cudaError_t e = cudaFuncSetAttribute(vs_est_tc_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, C1::kSmem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(vs_est_tc_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  e = cudaFuncSetAttribute(vs_est_tc_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, C2::kSmem);
   if (e != cudaSuccess) return e;
   const dim3 grid(nchunks, p.nh, p.B);
-  vs_est_tc_kernel<D, 1><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, p, tpc, nchunks);
+  vs_est_tc_kernel<D, 1><<<grid, C1::kThreads, C1::kSmem, stream>>>(tq, tk, p, tpc, nchunks);
   e = vs_combine_launch(p, nchunks, stream);
   if (e != cudaSuccess) return e;
-  vs_est_tc_kernel<D, 2><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, p, tpc, nchunks);
+  vs_est_tc_kernel<D, 2><<<grid, C2::kThreads, C2::kSmem, stream>>>(tq, tk, p, tpc, nchunks);
   // the tile's score rows are the last 64 query rows (rows beyond last_q are
   // zero), so the diagonal partials use the 64-row geometry
   VsEstParams q64 = p;
