@@ -188,7 +188,7 @@ minf_status attn_launch(const minf_shape* s, AttnParams& p, void* stream) {
 }
 
 bool vs_index_ok(const minf_vs_index* idx) {
-  return idx && idx->tgrp && idx->tgrp_cnt && idx->wmap && idx->vcnt && idx->vidx;
+  return idx && idx->tgrp && idx->tgrp_cnt && idx->wmap && idx->vcnt && idx->vidx && idx->tvcnt && idx->tvidx;
 }
 
 void set_vs_index(AttnParams& p, const minf_shape* s, const minf_vs_index* idx, int k_v, int k_s) {
@@ -197,6 +197,8 @@ void set_vs_index(AttnParams& p, const minf_shape* s, const minf_vs_index* idx, 
   p.wmap = idx->wmap;
   p.vcnt = idx->vcnt;
   p.vidx = idx->vidx;
+  p.tvcnt = idx->tvcnt;
+  p.tvidx = idx->tvidx;
   p.k_s = k_s;
   p.k_v = k_v;
   p.wmap_words = (int)minf_vs_wmap_words(s->N);
@@ -346,9 +348,11 @@ minf_status minf_build_index(const minf_shape* s, int nh, const int32_t* v_idx, 
   minf_status st = check_shape(s);
   if (st != MINF_OK) return st;
   if (!v_idx || !s_idx || !idx || !ws || nh < 1) return MINF_ERR_INVALID_ARG;
-  if (!idx->grp || !idx->grp_cnt || !idx->tgrp || !idx->tgrp_cnt || !idx->wmap || !idx->vcnt || !idx->vidx)
+  if (!idx->grp || !idx->grp_cnt || !idx->tgrp || !idx->tgrp_cnt || !idx->wmap || !idx->vcnt || !idx->vidx ||
+      !idx->tvcnt || !idx->tvidx)
     return MINF_ERR_INVALID_ARG;
   if (k_v < 1 || k_s < 1 || k_v > s->N || k_s > s->N) return MINF_ERR_INVALID_ARG;
+  if (s->N > (1 << 30)) return MINF_ERR_UNSUPPORTED;  // tvidx keeps the key in 30 bits
   if (ws_bytes < kStatusBytes) return MINF_ERR_WORKSPACE_TOO_SMALL;
   VsIndexParams p;
   p.v_idx = v_idx;

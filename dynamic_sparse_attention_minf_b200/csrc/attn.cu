@@ -178,30 +178,15 @@ struct Producer {
   int t;        // tiles whose K side (and descriptor) has been emitted
   int tv;       // tiles whose V side has been emitted: t - 1 (a range tile's V lags) or t
   int vj0[2];   // key chunks of tile tv while its V lags
-  int pend_k, pend_v;  // K and V slots of the gathered tile whose copies are issued but not yet signalled
   volatile int* abort;
   DevStatus* st;
   bool ok;
-
-  __device__ void flush_pending() {
-    if (pend_k >= 0) {
-      cp_async_wait<0>();
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&k_full[pend_k]);
-        mbar_arrive(&v_full[pend_v]);
-      }
-      pend_k = pend_v = -1;
-    }
-  }
 
   // Claims the K slot and the descriptor of tile t: S = Q K^T of tile t - S
   // is done and the softmax warps have read its descriptor.  False on abort.
   __device__ bool acquire_k(int& stage) {
     stage = t % C::kKStages;
     if (t >= C::kKStages) {
-      flush_pending();
       const uint32_t par = ((t / C::kKStages) - 1) & 1;
       if (!warp_wait(&k_empty[stage], par, abort, st, 1) || !warp_wait(&d_empty[stage], par, abort, st, 14)) {
         ok = false;
@@ -215,7 +200,6 @@ struct Producer {
   __device__ bool acquire_v(int u, int& stage) {
     stage = u % C::kVStages;
     if (u >= C::kVStages) {
-      flush_pending();
       if (!warp_wait(&v_empty[stage], ((u / C::kVStages) - 1) & 1, abort, st, 15)) {
         ok = false;
         return false;
@@ -311,43 +295,47 @@ struct Producer {
       dd.flags = F_MASK | (any_late ? F_CAUSAL : 0);
     }
     __syncwarp();
+    // 128 K rows, then 128 V rows, by cp.async into the 128B-swizzled layout.
+    // Every lane's copies lower the slot barrier's count when they land
+    // (cp.async.mbarrier.arrive), and lane 0's plain arrival completes the
+    // phase, so the producer never waits for a gather; the issuer adds the
+    // proxy fence that the generic-proxy writes need before the MMAs.
+    constexpr int CH = D * 2 / 16;  // 16-byte chunks per row
+    {
+      const uint32_t kb = smem_u32(smem + C::kOffK + stage * C::kKVBytes);
+#pragma unroll 8
+      for (int it = 0; it < 128 * CH / 32; ++it) {
+        const int idx = it * 32 + lane;
+        const int c = idx / CH, q = idx % CH;
+        const uint32_t off = (q >> 3) * C::kRegion + c * 128 + (((q & 7) ^ (c & 7)) << 4);
+        cp_async16(kb + off, Kh + (size_t)dd.cols[c] * D + q * 8);
+      }
+      cp_async_mbar_arrive(&k_full[stage]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&k_full[stage]);
+    }
     emit_v_lag();  // V of the previous tile
     int vstage;
     if (!acquire_v(t, vstage)) return;
-    // cp.async gather of 128 K and V rows into the 128B-swizzled layout.
-    constexpr int CH = D * 2 / 16;  // 16-byte chunks per row
-    const uint32_t kb = smem_u32(smem + C::kOffK + stage * C::kKVBytes);
-    const uint32_t vb = smem_u32(smem + C::kOffV + vstage * C::kKVBytes);
-#pragma unroll 4
-    for (int it = 0; it < 128 * CH / 32; ++it) {
-      const int idx = it * 32 + lane;
-      const int c = idx / CH;
-      const int q = idx % CH;
-      const int j = dd.cols[c];
-      const uint32_t off = (q >> 3) * C::kRegion + c * 128 + (((q & 7) ^ (c & 7)) << 4);
-      cp_async16(kb + off, Kh + (size_t)j * D + q * 8);
-      cp_async16(vb + off, Vh + (size_t)j * D + q * 8);
-    }
-    cp_async_commit();
-    // signal the previous gathered tile, keep this one in flight
-    if (pend_k >= 0) {
-      cp_async_wait<1>();
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&k_full[pend_k]);
-        mbar_arrive(&v_full[pend_v]);
+    {
+      const uint32_t vb = smem_u32(smem + C::kOffV + vstage * C::kKVBytes);
+#pragma unroll 8
+      for (int it = 0; it < 128 * CH / 32; ++it) {
+        const int idx = it * 32 + lane;
+        const int c = idx / CH, q = idx % CH;
+        const uint32_t off = (q >> 3) * C::kRegion + c * 128 + (((q & 7) ^ (c & 7)) << 4);
+        cp_async16(vb + off, Vh + (size_t)dd.cols[c] * D + q * 8);
       }
+      cp_async_mbar_arrive(&v_full[vstage]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&v_full[vstage]);
     }
-    pend_k = stage;
-    pend_v = vstage;
     ++t;
     ++tv;
   }
 
   __device__ void emit_end() {
     emit_v_lag();
-    flush_pending();
     if (!ok) return;
     int stage;
     if (!acquire_k(stage)) return;
@@ -411,6 +399,11 @@ struct Producer {
   }
 };
 
+// batches of 32 vertical-list entries whose loads are issued together
+constexpr int kVB = 8;
+// band tiles between two gathered tiles of a Vertical-Slash query tile
+constexpr int kGatherGap = 24;
+
 template <int D>
 __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int POL, int nh, int b, int hi, int qt) {
   const int R = qt * 128;
@@ -442,6 +435,48 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int POL, int 
     const int* tg = p.tgrp + hrow * p.k_s * 2;
     const int G = p.tgrp_cnt[hrow];
     const uint32_t* W = p.wmap + hrow * p.wmap_words;
+    // The tile's gathered columns come from its gather list, 128 per tile,
+    // one gathered tile after every kGatherGap band tiles (their copies take
+    // the producer several band tiles' time) and the rest after the bands.
+    // Each tile's list entries are loaded while the tile before is emitted.
+    const int nt = p.N / 128;
+    const int32_t* gl = p.tvidx + (hrow * nt + qt) * (size_t)p.k_v;
+    const int gcnt = min(__ldg(p.tvcnt + hrow * nt + qt), p.k_v);
+    int gpos = 0, since = 0;
+    uint32_t gbuf[4];
+    auto gload = [&]() {
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) {
+        const int c = gpos + 32 * wd + lane;
+        gbuf[wd] = (c < gcnt) ? (uint32_t)__ldg(gl + c) : 0u;
+      }
+    };
+    auto gemit = [&]() {
+      const int cnt = min(128, gcnt - gpos);
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) {
+        const int c = 32 * wd + lane;
+        if (c < cnt) {
+          int j = (int)(gbuf[wd] & 0x3FFFFFFFu);
+          if (j > R + 127) { report(P.st, MINF_ERR_DEVICE_BOUNDS, 20); j = 0; }
+          P.scols[c] = j;
+          P.sbits[c] = (uint8_t)(gbuf[wd] >> 30);
+        }
+      }
+      __syncwarp();
+      P.emit_gather(cnt);
+      __syncwarp();
+      gpos += cnt;
+      gload();
+    };
+    auto band = [&](int j0, uint32_t word, int flags) {
+      P.emit_range(j0, j0 + 64, word, flags);
+      if (++since == kGatherGap) {
+        since = 0;
+        if (gpos < gcnt && P.ok) gemit();
+      }
+    };
+    gload();
     // Slash bands, in ascending keys = descending offsets.  Only tile groups
     // with a_G <= R + 127 reach this query tile: binary-search the last one,
     // then walk down 32 groups at a time, one group per lane, each lane
@@ -500,7 +535,7 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int POL, int 
         uint32_t wnext = (ntile > 5) ? chunk_word(1) : 0xFFFFFFFFu;
         {
           const int cnt = min(128, hi_key - lo_key + 1);
-          P.emit_range(lo_key, lo_key + 64, wf, (lo_key + cnt - 1 > R) ? F_CAUSAL : 0);
+          band(lo_key, wf, (lo_key + cnt - 1 > R) ? F_CAUSAL : 0);
         }
         for (int tt = 1; tt < ntile && P.ok; ++tt) {
           const int slot = (tt - 1) & 3;
@@ -512,33 +547,11 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int POL, int 
           const uint32_t wv = __shfl_sync(0xFFFFFFFFu, wcur, slot * 8 + (lane & 7));
           const int j0 = lo_key + 128 * tt;
           const int cnt = min(128, hi_key - j0 + 1);
-          P.emit_range(j0, j0 + 64, lane < 8 ? wv : 0xFFFFFFFFu, (j0 + cnt - 1 > R) ? F_CAUSAL : 0);
+          band(j0, lane < 8 ? wv : 0xFFFFFFFFu, (j0 + cnt - 1 > R) ? F_CAUSAL : 0);
         }
       }
     }
-    // verticals: V_{b1} (both halves as applicable), then V_{b0} on half-1 bands
-    const int nb = p.N / 64;
-    const int b0 = R / 64, b1 = b0 + 1;
-    const int* vl1 = p.vidx + (hrow * nb + b1) * (size_t)p.k_v;
-    const int* vl0 = p.vidx + (hrow * nb + b0) * (size_t)p.k_v;
-    const int c1 = min(p.vcnt[hrow * nb + b1], p.k_v);
-    const int c0 = min(p.vcnt[hrow * nb + b0], p.k_v);
-    int n_staged = 0;
-    for (int base = 0; base < c1 && P.ok; base += 32) {
-      const int idx = base + lane;
-      int j = (idx < c1) ? vl1[idx] : 0;
-      if (j < 0 || j > R + 127) { if (idx < c1) report(P.st, MINF_ERR_DEVICE_BOUNDS, 20); j = 0; }
-      const uint32_t h0 = (idx < c1 && j <= R + 63 && !wmap_bit(W, R - j + 63)) ? 1u : 0u;
-      P.append(idx < c1, j, h0 | 2u, n_staged);
-    }
-    for (int base = 0; base < c0 && P.ok; base += 32) {
-      const int idx = base + lane;
-      int j = (idx < c0) ? vl0[idx] : 0;
-      if (j < 0 || j > R + 63) { if (idx < c0) report(P.st, MINF_ERR_DEVICE_BOUNDS, 21); j = 0; }
-      const bool keep = (idx < c0) && wmap_bit(W, R + 127 - j);
-      P.append(keep, j, 1u, n_staged);
-    }
-    if (n_staged > 0 && P.ok) P.emit_gather(n_staged);
+    while (gpos < gcnt && P.ok) gemit();
   } else if (POL == POL_VS_EXACT) {
     // The same key ranges as the band variant at 128-row granularity (one per
     // offset group of gap 128), masked element by element by the softmax from
@@ -577,11 +590,21 @@ __device__ void produce_tiles(Producer<D>& P, const AttnParams& p, int POL, int 
     const int* vl = p.vidx + (hrow * nt + qt) * (size_t)p.k_v;
     const int c = min(p.vcnt[hrow * nt + qt], p.k_v);
     int n_staged = 0;
-    for (int base = 0; base < c && P.ok; base += 32) {
-      const int idx = base + lane;
-      int j = (idx < c) ? vl[idx] : 0;
-      if (j < 0 || j > R + 127) { if (idx < c) report(P.st, MINF_ERR_DEVICE_BOUNDS, 24); j = 0; }
-      P.append(idx < c, j, (j <= R + 63 ? 1u : 0u) | 2u, n_staged);
+    for (int base = 0; base < c && P.ok; base += 32 * kVB) {
+      int jv[kVB];
+#pragma unroll
+      for (int k = 0; k < kVB; ++k) {
+        const int idx = base + 32 * k + lane;
+        jv[k] = (idx < c) ? __ldg(vl + idx) : 0;
+      }
+#pragma unroll
+      for (int k = 0; k < kVB; ++k) {
+        if (base + 32 * k >= c || !P.ok) break;
+        const int idx = base + 32 * k + lane;
+        int j = jv[k];
+        if (j < 0 || j > R + 127) { if (idx < c) report(P.st, MINF_ERR_DEVICE_BOUNDS, 24); j = 0; }
+        P.append(idx < c, j, (j <= R + 63 ? 1u : 0u) | 2u, n_staged);
+      }
     }
     if (n_staged > 0 && P.ok) P.emit_gather(n_staged);
   } else if (POL == POL_BS) {
@@ -762,7 +785,6 @@ __global__ void __launch_bounds__(320, 1)
     P.t = 0;
     P.tv = 0;
     P.vj0[0] = P.vj0[1] = 0;
-    P.pend_k = P.pend_v = -1;
     P.abort = abort;
     P.st = p.status;
     P.ok = true;
@@ -786,7 +808,6 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0 && P.ok) atomicAdd(&p.status->tiles, (unsigned long long)P.t);
       P.emit_end();
     }
-    P.flush_pending();
     P.drain();
     if (lane == 0) {
       int dummy = 0;
@@ -799,11 +820,12 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t qaddr = smem_u32(smem + C::kOffQ);
     // O_0 += P[:, 0:64] V[0:64, :] and O_1 += P[:, 64:128] V[64:128, :];
     // warpgroup w's bf16 P occupies TMEM columns 64w .. 64w+31 of the buffer
-    auto issue_pv = [&](int tp) -> bool {
+    auto issue_pv = [&](int tp, bool gathered) -> bool {
       const int bp = tp & 1;
       const int sp = tp % C::kVStages;
       if (!warp_wait(&p_full[bp], (tp >> 1) & 1, abort, p.status, 3)) return false;
       if (!warp_wait(&v_full[sp], (tp / C::kVStages) & 1, abort, p.status, 4)) return false;
+      if (gathered) fence_proxy_async();  // V rows written by cp.async
       tc_fence_after();
       // descriptors of the K-steps: the stage's base plus a constant (the
       // start-address field holds address / 16 and never carries out)
@@ -825,13 +847,18 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = warp_wait(q_full, 0, abort, p.status, 2);
     const uint64_t qd0 = sdesc_sw128(qaddr, 16, 1024);
     int t = 0, pend = -1;
+    bool pend_gathered = false;
     while (ok) {
       const int st = t % C::kKStages;
       if (!warp_wait(&k_full[st], (t / C::kKStages) & 1, abort, p.status, 5)) { ok = false; break; }
-      if (__all_sync(0xFFFFFFFFu, desc[st].kind == KIND_END)) break;
-      // Q and K were written by TMA or by cp.async plus the producer's proxy
-      // fence; the barrier alone orders them before the MMA (no tcgen05
-      // fence here: it would stall the issue of every tile).
+      const int kd = desc[st].kind;
+      if (__all_sync(0xFFFFFFFFu, kd == KIND_END)) break;
+      // Q and range K tiles were written by TMA, and the barrier alone orders
+      // them before the MMA (no tcgen05 fence here: it would stall the issue
+      // of every tile); gathered rows were written by cp.async, whose
+      // generic-proxy writes need a proxy fence first.
+      const bool gathered = __all_sync(0xFFFFFFFFu, kd == KIND_GATHER);
+      if (gathered) fence_proxy_async();
       const int w = t & 1;  // S buffer
       const uint64_t kd0 = sdesc_sw128(smem_u32(smem + C::kOffK + st * C::kKVBytes), 16, 1024);
       if (elect_one()) {
@@ -844,11 +871,12 @@ __global__ void __launch_bounds__(320, 1)
         umma_commit(&k_empty[st]);
       }
       __syncwarp();
-      if (pend >= 0 && !issue_pv(pend)) { ok = false; pend = -1; break; }
+      if (pend >= 0 && !issue_pv(pend, pend_gathered)) { ok = false; pend = -1; break; }
       pend = t;
+      pend_gathered = gathered;
       ++t;
     }
-    if (ok && pend >= 0) issue_pv(pend);
+    if (ok && pend >= 0) issue_pv(pend, pend_gathered);
     if (elect_one()) umma_commit(mma_done);
     __syncwarp();
     if (lane == 0) {

@@ -38,14 +38,17 @@ struct AttnParams {
   float scale_log2;  // softmax scale * log2(e)
   // A-shape
   int n_sink, n_local;
-  // Vertical-Slash index (band reading: tgrp, wmap, per-64-row-block vcnt /
-  // vidx; exact reading: tgrp, twmap, sbits, vbits, per-128-row-tile lists)
+  // Vertical-Slash index (band reading: tgrp, wmap, per-128-row-tile gather
+  // lists tvcnt / tvidx; exact reading: tgrp, twmap, sbits, vbits,
+  // per-128-row-tile lists vcnt / vidx)
   const int32_t* tgrp;
   const int32_t* tgrp_cnt;
   const uint32_t* wmap;
   const uint32_t* twmap;
   const int32_t* vcnt;
   const int32_t* vidx;
+  const int32_t* tvcnt;
+  const int32_t* tvidx;
   int k_s, k_v, wmap_words, twmap_words;
   const uint32_t* sbits;
   const uint32_t* vbits;

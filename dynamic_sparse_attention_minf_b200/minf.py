@@ -41,7 +41,7 @@ class Shape(ctypes.Structure):
 
 class _VsIndexC(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("grp", "grp_cnt", "tgrp", "tgrp_cnt", "wmap", "vcnt", "vidx")]
+                ("grp", "grp_cnt", "tgrp", "tgrp_cnt", "wmap", "vcnt", "vidx", "tvcnt", "tvidx")]
 
 
 class _VsExactIndexC(ctypes.Structure):
@@ -141,6 +141,8 @@ class VSIndex:
     wmap: torch.Tensor
     vcnt: torch.Tensor
     vidx: torch.Tensor
+    tvcnt: torch.Tensor
+    tvidx: torch.Tensor
     k_v: int
     k_s: int
 
@@ -151,11 +153,12 @@ class VSIndex:
         return VSIndex(torch.empty(B, nh, k_s, 2, **i32), torch.empty(B, nh, **i32),
                        torch.empty(B, nh, k_s, 2, **i32), torch.empty(B, nh, **i32),
                        torch.empty(B, nh, W, **i32), torch.empty(B, nh, N // 64, **i32),
-                       torch.empty(B, nh, N // 64, k_v, **i32), k_v, k_s)
+                       torch.empty(B, nh, N // 64, k_v, **i32), torch.empty(B, nh, N // 128, **i32),
+                       torch.empty(B, nh, N // 128, k_v, **i32), k_v, k_s)
 
     def c(self):
         return _VsIndexC(*(t.data_ptr() for t in (self.grp, self.grp_cnt, self.tgrp, self.tgrp_cnt,
-                                                  self.wmap, self.vcnt, self.vidx)))
+                                                  self.wmap, self.vcnt, self.vidx, self.tvcnt, self.tvidx)))
 
 
 # ----------------------------------------------------------------- entry points

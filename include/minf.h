@@ -101,6 +101,15 @@ enum {
  *   vcnt     [B, nh, nb]     per 64-row query block, the number of vertical
  *                            columns not already covered by a slash band
  *   vidx     [B, nh, nb, k_v] those columns, ascending (j <= last row of the block)
+ *   tvcnt    [B, nh, nt]      per 128-row query tile (nt = N / 128, blocks 2t and
+ *                            2t + 1), the number of entries of tvidx
+ *   tvidx    [B, nh, nt, k_v] the columns the tile gathers, each with its rows:
+ *                            key j in bits 0-29, bit 30 set iff block 2t lists
+ *                            j, bit 31 iff block 2t + 1 does.  First block
+ *                            2t + 1's list in order, then the columns of block
+ *                            2t's list that block 2t + 1 does not list.  Every
+ *                            column of V appears at most once per tile, so k_v
+ *                            entries suffice.  Requires N <= 2^30.
  */
 typedef struct {
   int32_t* grp;
@@ -110,6 +119,8 @@ typedef struct {
   uint32_t* wmap;
   int32_t* vcnt;
   int32_t* vidx;
+  int32_t* tvcnt;
+  int32_t* tvidx;
 } minf_vs_index;
 
 /* Number of 32-bit words of one head's slash-band bitmap (wmap). */

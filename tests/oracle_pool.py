@@ -14,7 +14,7 @@ from multiprocessing import shared_memory
 import numpy as np
 
 from oracle import minf_oracle as orc
-from tests.parity import GAP, LSE_ABS, MAX_ABS, MEAN_ABS
+from tests.parity import GAP, LSE_ABS, MAX_ABS, MEAN_ABS, tile_list_errors
 
 
 @dataclass
@@ -113,6 +113,11 @@ def check_head(task: dict) -> dict:
                 bad = [b for b in range(N // 64) if not np.array_equal(VI[task["slot"], b, :vcnt[b]], vidx[b, :vcnt[b]])]
                 if bad:
                     out["errors"].append(f"vidx differs in {len(bad)} blocks, e.g. {bad[:4]}")
+            if "tvidx" in task:
+                s_tv, TV = task["tvidx"].attach(); shms.append(s_tv)
+                bad = tile_list_errors(task["tvcnt"], TV[task["slot"]], vcnt, vidx)
+                if bad:
+                    out["errors"].append(f"tile gather lists differ in {len(bad)} tiles, e.g. {bad[:4]}")
             mask_fn = lambda r: orc.mask_vs(r, N, gv, gs)
             if "ox_rows" in task:
                 # element-exact variant on the same sets: its per-tile vertical

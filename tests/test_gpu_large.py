@@ -63,6 +63,8 @@ def test_full_size_layer(cid):
         if vs_pos:
             idx = b["vs_index"]
             VI = op.share(idx.vidx[0].cpu().numpy(), keep)
+            TV = op.share(idx.tvidx[0].cpu().numpy(), keep)
+            tvcnt = idx.tvcnt[0].cpu().numpy()
             v_idx, s_idx = b["v_idx"][0].cpu().numpy(), b["s_idx"][0].cpu().numpy()
             grp, grp_cnt = idx.grp[0].cpu().numpy(), idx.grp_cnt[0].cpu().numpy()
             tgrp, tgrp_cnt = idx.tgrp[0].cpu().numpy(), idx.tgrp_cnt[0].cpu().numpy()
@@ -79,6 +81,7 @@ def test_full_size_layer(cid):
                 a = vs_pos[h]
                 t.update(pattern="vs", k_v=w.k_v, k_s=w.k_s, v_idx=v_idx[a], s_idx=s_idx[a],
                          grp=grp[a, :grp_cnt[a]], tgrp=tgrp[a, :tgrp_cnt[a]], vcnt=vcnt[a], vidx=VI, slot=a,
+                         tvcnt=tvcnt[a], tvidx=TV,
                          ox_rows=ox_rows[h], lsex_rows=lsex_rows[h], xcnt=xcnt[a], xidx=XI)
             elif h in bs_pos:
                 a = bs_pos[h]

@@ -8,7 +8,7 @@ import torch
 from dynamic_sparse_attention_minf_b200 import minf
 from dynamic_sparse_attention_minf_b200 import workloads as wl
 from oracle import minf_oracle as orc
-from tests.parity import check_close, check_index_set, check_lse
+from tests.parity import check_close, check_index_set, check_lse, tile_list_errors
 
 pytestmark = pytest.mark.gpu
 
@@ -100,6 +100,8 @@ def _vs_pipeline(w, heads, rows=None):
         gvi = index.vidx[0, hi].cpu().numpy()
         for b in range(w.N // 64):
             assert np.array_equal(gvi[b, :vcnt[b]], vidx[b, :vcnt[b]]), f"block {b}"
+        bad = tile_list_errors(index.tvcnt[0, hi].cpu().numpy(), index.tvidx[0, hi].cpu().numpy(), vcnt, vidx)
+        assert not bad, f"tile gather lists differ in tiles {bad[:4]}"
     _check_attn(o, lse, qn, kn, vn, heads, w,
                 lambda hi, h: (lambda r: orc.mask_vs(r, w.N, gv[hi], gs[hi])), rows)
     return gv, gs
