@@ -122,8 +122,11 @@ size_t plan_vs_est(const minf_shape* s, int nh, char* ws, VsEstWs* out) {
 struct BsEstWs {
   DevStatus* status;
   float *qbar, *kbar, *scores;
+  __nv_bfloat16 *qs, *ks;
 };
-size_t plan_bs_est(const minf_shape* s, int nh, char* ws, BsEstWs* out) {
+// The pooled means and the pooled score matrix; with a budget k_b that the
+// tensor-core path takes (k_b = 0 never), also the means' bf16 parts.
+size_t plan_bs_est(const minf_shape* s, int nh, int k_b, char* ws, BsEstWs* out) {
   Carver c{ws, 0};
   const size_t bh = (size_t)s->B * nh;
   const size_t nb = s->N / 64;
@@ -132,8 +135,44 @@ size_t plan_bs_est(const minf_shape* s, int nh, char* ws, BsEstWs* out) {
   w.qbar = c.take<float>(bh * nb * s->d);
   w.kbar = c.take<float>(bh * nb * s->d);
   w.scores = c.take<float>(bh * nb * nb);
+  w.qs = w.ks = nullptr;
+  if (bs_select_supported(s->N, s->d, k_b)) {
+    w.qs = c.take<__nv_bfloat16>(3 * bh * nb * s->d);
+    w.ks = c.take<__nv_bfloat16>(3 * bh * nb * s->d);
+  }
   if (out) *out = w;
   return c.off;
+}
+
+// 3-D bf16 view of the split key means [3 * bh, nb, d]: x = d, y = key block,
+// z = part * bh + slot, with 64 x 128 x 1 boxes (128-byte swizzled); rows
+// past nb read as zero.
+// 3-D fp32 view of the pooled score matrices [bh, nb, nb]: x = key block,
+// y = query block, z = slot, with 32 x 128 x 1 boxes (128-byte swizzled).
+bool make_scores_map(CUtensorMap* m, const void* ptr, long long bh, int nb) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)nb, (cuuint64_t)nb, (cuuint64_t)bh};
+  cuuint64_t strides[2] = {(cuuint64_t)nb * 4, (cuuint64_t)nb * nb * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_parts_map(CUtensorMap* m, const void* ptr, long long bh, int nb, int d) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)nb, (cuuint64_t)(3 * bh)};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)nb * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 // Checks the arguments every attention call shares and fills the common
@@ -221,7 +260,7 @@ size_t minf_workspace_size(int op, const minf_shape* s, int nh, int k_v, int k_s
     case MINF_OP_ESTIMATE_VS:
       return plan_vs_est(s, nh, nullptr, nullptr);
     case MINF_OP_ESTIMATE_BS:
-      return plan_bs_est(s, nh, nullptr, nullptr);
+      return plan_bs_est(s, nh, k_b, nullptr, nullptr);
     case MINF_OP_BUILD_INDEX:
     case MINF_OP_BUILD_INDEX_EXACT:
     case MINF_OP_SPARSE_ATTN_VS_EXACT:
@@ -304,9 +343,11 @@ minf_status minf_estimate_bs(const minf_shape* s, const minf_bf16* Q, const minf
   if (!Q || !K || !heads || !blk_idx || !blk_cnt || !ws) return MINF_ERR_INVALID_ARG;
   if (nh < 1 || nh > s->Hq || k_b < 1) return MINF_ERR_INVALID_ARG;
   if (block != 64) return MINF_ERR_UNSUPPORTED;
-  if (ws_bytes < plan_bs_est(s, nh, nullptr, nullptr)) return MINF_ERR_WORKSPACE_TOO_SMALL;
+  // the tensor-core path, unless the workspace was sized without it (k_b = 0)
+  const bool fused = bs_select_supported(s->N, s->d, k_b) && ws_bytes >= plan_bs_est(s, nh, k_b, nullptr, nullptr);
+  if (!fused && ws_bytes < plan_bs_est(s, nh, 0, nullptr, nullptr)) return MINF_ERR_WORKSPACE_TOO_SMALL;
   BsEstWs w;
-  plan_bs_est(s, nh, (char*)ws, &w);
+  plan_bs_est(s, nh, fused ? k_b : 0, (char*)ws, &w);
   BsEstParams p;
   p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
   p.K = reinterpret_cast<const __nv_bfloat16*>(K);
@@ -322,11 +363,24 @@ minf_status minf_estimate_bs(const minf_shape* s, const minf_bf16* Q, const minf
   p.qbar = w.qbar;
   p.kbar = w.kbar;
   p.scores = blk_score ? blk_score : w.scores;
+  p.qs = fused ? w.qs : nullptr;
+  p.ks = fused ? w.ks : nullptr;
   p.status = w.status;
   cudaStream_t cs = (cudaStream_t)stream;
+  const int nb = s->N / 64;
+  if (fused) {
+    CUtensorMap tm, tms;
+    if (!make_parts_map(&tm, w.ks, (long long)s->B * nh, nb, s->d) ||
+        !make_scores_map(&tms, p.scores, (long long)s->B * nh, nb))
+      return MINF_ERR_CUDA;
+    BsEstParams pool = p;
+    pool.scores = nullptr;  // pooling and split only
+    cudaError_t e = bs_pool_score_launch(pool, cs);
+    if (e != cudaSuccess) return MINF_ERR_CUDA;
+    return cuda_status(bs_select_launch(tm, tms, p, k_b, blk_idx, blk_cnt, cs));
+  }
   cudaError_t e = bs_pool_score_launch(p, cs);
   if (e != cudaSuccess) return MINF_ERR_CUDA;
-  const int nb = s->N / 64;
   TopkRows t;
   t.scores = p.scores;
   t.row_stride = nb;

@@ -627,8 +627,22 @@ __global__ void bs_pool_kernel(const BsEstParams p) {
                                  : p.Q + ((size_t)(b * p.Hq + head) * p.N + qb * 64) * p.d;
   float s = 0.f;
   for (int r = 0; r < 64; ++r) s += __bfloat162float(src[(size_t)r * p.d + dd]);
-  float* dst = (isk ? p.kbar : p.qbar) + (((size_t)(b * p.nh + hi) * nb) + qb) * p.d;
-  dst[dd] = s * (1.0f / 64.0f);
+  const size_t at = (((size_t)(b * p.nh + hi) * nb) + qb) * p.d + dd;
+  const float m = s * (1.0f / 64.0f);
+  (isk ? p.kbar : p.qbar)[at] = m;
+  __nv_bfloat16* parts = isk ? p.ks : p.qs;
+  if (parts) {
+    // m = x0 + x1 + x2 up to 2^-24 relative: each part is the bf16 rounding
+    // of what the earlier parts leave, and every difference is exact in fp32
+    const size_t stride = (size_t)p.B * p.nh * nb * p.d;
+    const __nv_bfloat16 x0 = __float2bfloat16_rn(m);
+    const float r1 = m - __bfloat162float(x0);
+    const __nv_bfloat16 x1 = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(x1);
+    parts[at] = x0;
+    parts[stride + at] = x1;
+    parts[2 * stride + at] = __float2bfloat16_rn(r2);
+  }
 }
 
 // t[b, c] = scale * qbar_b . kbar_c over 64 x 64 tiles with c-tile <= b-tile.
@@ -761,6 +775,7 @@ __global__ void __launch_bounds__(256) bs_score_tri_kernel(const BsEstParams p, 
 cudaError_t bs_pool_score_launch(const BsEstParams& p, cudaStream_t stream) {
   const int nb = p.N / 64;
   bs_pool_kernel<<<dim3(nb, p.nh, p.B), 2 * p.d, 0, stream>>>(p);
+  if (!p.scores) return cudaGetLastError();
   if (nb % 8 == 0 && p.d % kBsK == 0) {
     const int nt = (nb + kBsT - 1) / kBsT;
     bs_score_tri_kernel<<<dim3(nt * (nt + 1) / 2, p.B * p.nh), 256, 0, stream>>>(p, nt);

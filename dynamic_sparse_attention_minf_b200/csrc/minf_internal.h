@@ -117,9 +117,24 @@ struct BsEstParams {
   float* qbar;     // [B, nh, nb, d]
   float* kbar;     // [B, nh, nb, d]
   float* scores;   // [B, nh, nb, nb]
+  __nv_bfloat16* qs;  // [3, B, nh, nb, d]: qbar = qs[0] + qs[1] + qs[2] (bf16 parts), or NULL
+  __nv_bfloat16* ks;  // [3, B, nh, nb, d], the same for kbar
   DevStatus* status;
 };
+// Pools Q and K per 64-row block (and splits the means into bf16 parts when
+// qs / ks are set); when `scores` is set, also writes the pooled score matrix.
 cudaError_t bs_pool_score_launch(const BsEstParams& p, cudaStream_t stream);
+
+// Block-Sparse selection fused with the pooled scores on the tensor cores
+// (bs_select.cu): from the split means, the k best key blocks of every query
+// block, diagonal forced, in ascending order.
+// tmKs: the key parts as a 3-D bf16 view (x = d, y = key block, z = part *
+// B * nh + batch * nh + head slot) with 64 x 128 x 1 boxes; tmS: the score
+// matrices as a 3-D fp32 view (x = key block, y = query block, z = batch * nh
+// + head slot) with 32 x 128 x 1 boxes; both 128-byte swizzled.
+bool bs_select_supported(int N, int d, int k);
+cudaError_t bs_select_launch(const CUtensorMap& tmKs, const CUtensorMap& tmS, const BsEstParams& p, int k,
+                             int32_t* blk_idx, int32_t* blk_cnt, cudaStream_t stream);
 
 struct VsIndexParams {
   const int32_t* v_idx;

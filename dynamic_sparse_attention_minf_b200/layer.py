@@ -75,7 +75,7 @@ def make_plan(w: Workload, device="cuda") -> LayerPlan:
         nbh = len(bs)
         plan.bufs["blk_idx"] = torch.empty(B, nbh, N // 64, w.k_b, **i32)
         plan.bufs["blk_cnt"] = torch.empty(B, nbh, N // 64, **i32)
-        plan.bufs["ws_bs_est"] = minf.workspace(minf.OP_ESTIMATE_BS, shp, nbh, device=dev)
+        plan.bufs["ws_bs_est"] = minf.workspace(minf.OP_ESTIMATE_BS, shp, nbh, k_b=w.k_b, device=dev)
         plan.bufs["ws_bs_attn"] = minf.workspace(minf.OP_SPARSE_ATTN_BS, shp, nbh, device=dev)
     if ah:
         plan.a_heads = torch.tensor(ah, **i32)

@@ -191,7 +191,7 @@ def minf_estimate_bs(q, k, heads, k_b, block=64, scale=0.0, return_scores=False,
     blk_cnt = torch.empty(shp.B, nh, nb, dtype=torch.int32, device=q.device)
     sc = torch.empty(shp.B, nh, nb, nb, dtype=torch.float32, device=q.device) if return_scores else None
     if ws is None:
-        ws = workspace(OP_ESTIMATE_BS, shp, nh, device=q.device)
+        ws = workspace(OP_ESTIMATE_BS, shp, nh, k_b=k_b, device=q.device)
     _check("minf_estimate_bs", lib().minf_estimate_bs(
         ctypes.byref(shp), _p(q), _p(k), _p(hd), nh, block, k_b, _p(blk_idx), _p(blk_cnt), _p(sc),
         _p(ws), ws.numel(), _stream(stream)))

@@ -130,6 +130,8 @@ size_t minf_vs_wmap_words(int N);
  * Bytes of workspace that operation `op` needs for this shape, head count and
  * budgets (k_v, k_s, k_b are ignored where the operation has none).  Always at
  * least 256 (the status word).  Returns 0 for an unknown op or a bad shape.
+ * MINF_OP_ESTIMATE_BS: the size for the fused selection when k_b allows it,
+ * else (k_b = 0 included) for the pooled score matrix.
  */
 size_t minf_workspace_size(int op, const minf_shape* shape, int nh, int k_v, int k_s, int k_b);
 
@@ -173,12 +175,20 @@ minf_status minf_estimate_vs_noalloc(const minf_shape* shape, const minf_bf16* Q
 
 /*
  * Block-Sparse index estimation (summary, "Key points": queries and keys are
- * mean-pooled in 64-token blocks).  Pooled means are taken in fp32 and the
- * pooled scores t[b, c] = scale * Qbar_b . Kbar_c (c <= b) are formed with fp32
- * FMAs; per query block b the k_b best key blocks are kept, block b itself
- * always.  block must be 64.  Outputs: blk_idx [B, nh, N/64, k_b] ascending,
- * padded with -1; blk_cnt [B, nh, N/64] = min(b + 1, k_b).  blk_score, when
- * non-NULL, receives t as [B, nh, N/64, N/64] (entries with c > b undefined).
+ * mean-pooled in 64-token blocks).  Pooled means are taken in fp32; per query
+ * block b the k_b best key blocks c <= b by the pooled score
+ * t[b, c] = scale * Qbar_b . Kbar_c are kept (ties to the lower c), block b
+ * itself always.  block must be 64.  Outputs: blk_idx [B, nh, N/64, k_b]
+ * ascending, padded with -1; blk_cnt [B, nh, N/64] = min(b + 1, k_b).
+ *
+ * For d = 128 and k_b <= 128, t is formed on the tensor cores from the means
+ * split into three bf16 parts each (six products per K step: fp32
+ * accuracy), and each row is selected by one warp from the diagonal down;
+ * this needs the workspace minf_workspace_size gives for this k_b.  Otherwise
+ * (or with a workspace sized for k_b = 0) t is formed with fp32 FMAs.  Either
+ * way t is stored as a [N/64, N/64] matrix per head; blk_score, when
+ * non-NULL, receives it as [B, nh, N/64, N/64] (entries with c > b
+ * undefined).
  */
 minf_status minf_estimate_bs(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K,
                              const int32_t* heads, int nh, int block, int k_b,

@@ -47,8 +47,15 @@ def test_workspace_sizes(L):
         assert L.minf_workspace_size(op, ctypes.byref(s), 24, 1000, 6096, 100) >= 256
     vs = L.minf_workspace_size(minf.OP_ESTIMATE_VS, ctypes.byref(s), 24, 1000, 6096, 0)
     assert vs >= 24 * 131072 * 4 * 2          # both score vectors
+    # Block-Sparse: the pooled means and score matrix; with a budget the
+    # tensor-core path takes (k_b = 100), also the means' three bf16 parts
+    base = 2 * 6 * 2048 * 128 * 4 + 6 * 2048 * 2048 * 4
+    parts = 2 * 3 * 6 * 2048 * 128 * 2
     bs = L.minf_workspace_size(minf.OP_ESTIMATE_BS, ctypes.byref(s), 6, 0, 0, 100)
-    assert bs >= 6 * 2048 * 2048 * 4          # pooled score matrix
+    assert bs >= base + parts
+    for kb in (0, 200):
+        bs0 = L.minf_workspace_size(minf.OP_ESTIMATE_BS, ctypes.byref(s), 6, 0, 0, kb)
+        assert base <= bs0 < base + parts
     bad = minf.Shape(1, 32, 8, 1000, 128, 0.0)
     assert L.minf_workspace_size(0, ctypes.byref(bad), 24, 1, 1, 1) == 0
     assert L.minf_workspace_size(99, ctypes.byref(s), 24, 1, 1, 1) == 0

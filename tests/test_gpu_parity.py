@@ -158,6 +158,13 @@ def _bs_pipeline(w, heads, rows=None):
     blk_idx, blk_cnt, t = minf.minf_estimate_bs(q, k, heads, w.k_b, return_scores=True, ws=ws)
     assert minf.minf_get_device_status(ws) == 0
     gi, gc = blk_idx[0].cpu().numpy(), blk_cnt[0].cpu().numpy()
+    # with a workspace sized for the budget (d = 128): scores on the tensor
+    # cores from the split means, one warp per row selecting; held to the
+    # same rules against the oracle
+    ws_f = minf.workspace(minf.OP_ESTIMATE_BS, minf.shape_of(q, k), len(heads), k_b=w.k_b)
+    fi, fc, tf = minf.minf_estimate_bs(q, k, heads, w.k_b, return_scores=True, ws=ws_f)
+    assert minf.minf_get_device_status(ws_f) == 0
+    fi, fc = fi[0].cpu().numpy(), fc[0].cpu().numpy()
     nb = w.N // 64
     flips = 0
     for hi, h in enumerate(heads):
@@ -167,11 +174,13 @@ def _bs_pipeline(w, heads, rows=None):
         tg = t[0, hi].cpu().numpy()
         low = np.tril(np.ones((nb, nb), bool))
         np.testing.assert_allclose(tg[low], tref[low], rtol=1e-4, atol=1e-5)
-        assert np.array_equal(gc[hi], rc)
-        for b in range(nb):
-            flips += check_index_set(gi[hi, b, :gc[hi, b]], ri[b, :rc[b]], tref[b, :b + 1], forced=b,
-                                     what=f"h{h} block {b}")
-            assert (gi[hi, b, gc[hi, b]:] == -1).all()
+        np.testing.assert_allclose(tf[0, hi].cpu().numpy()[low], tref[low], rtol=1e-4, atol=1e-5)
+        for xi, xc, how in ((gi, gc, "fp32 FMA"), (fi, fc, "tensor cores")):
+            assert np.array_equal(xc[hi], rc), how
+            for b in range(nb):
+                flips += check_index_set(xi[hi, b, :xc[hi, b]], ri[b, :rc[b]], tref[b, :b + 1], forced=b,
+                                         what=f"{how} h{h} block {b}")
+                assert (xi[hi, b, xc[hi, b]:] == -1).all(), how
     ws_a = minf.workspace(minf.OP_SPARSE_ATTN_BS, minf.shape_of(q, k), len(heads))
     o, lse = minf.minf_sparse_attn_bs(q, k, v, heads, blk_idx, blk_cnt, ws=ws_a)
     assert minf.minf_get_device_status(ws_a) == 0
@@ -191,6 +200,41 @@ def test_bs_config1_sampled_rows():
     w = wl.config(1)
     rows = wl.sample_rows(w.N, 512, w.seed).numpy()
     _bs_pipeline(w, list(range(8)), rows)
+
+
+@pytest.mark.parametrize("k_b", [1, 128])
+def test_bs_fused_selection_long_rows(k_b):
+    """The tensor-core path over several 128-block row tiles, at the largest
+    budget it takes (a row's candidate list compacts several times) and at
+    k_b = 1 (only the forced diagonal), against the oracle's selection."""
+    w = wl.small(Hq=2, Hkv=1, N=32768, d=128, seed=17, bias="block", patterns=[wl.PAT_BS] * 2, k_b=k_b)
+    q, k, v, qn, kn, vn = _inputs(w)
+    sc = orc.default_scale(w.d)
+    gi, gc = minf.minf_estimate_bs(q, k, [0, 1], k_b)
+    gi, gc = gi[0].cpu().numpy(), gc[0].cpu().numpy()
+    for h in range(2):
+        ri, rc = orc.bs_select(qn[h], kn[0], sc, k_b)
+        tref = orc.bs_scores(orc.bs_pool(qn[h]), orc.bs_pool(kn[0]), sc)
+        assert np.array_equal(gc[h], rc)
+        for b in range(w.N // 64):
+            check_index_set(gi[h, b, :gc[h, b]], ri[b, :rc[b]], tref[b, :b + 1], forced=b, what=f"h{h} block {b}")
+            assert (gi[h, b, gc[h, b]:] == -1).all()
+
+
+def test_bs_fused_selection_all_ties():
+    """Zero queries and keys: every pooled score ties, so each row keeps its
+    diagonal block and the lowest other blocks."""
+    N, k_b = 16384, 128
+    q = torch.zeros(1, 2, N, 128, dtype=torch.bfloat16, device=DEV)
+    k = torch.zeros(1, 1, N, 128, dtype=torch.bfloat16, device=DEV)
+    gi, gc = minf.minf_estimate_bs(q, k, [0, 1], k_b)
+    gi, gc = gi[0].cpu().numpy(), gc[0].cpu().numpy()
+    z = np.zeros((N, 128))
+    ri, rc = orc.bs_select(z, z, orc.default_scale(128), k_b)
+    for h in range(2):
+        assert np.array_equal(gc[h], rc)
+        for b in range(N // 64):
+            assert np.array_equal(gi[h, b, :gc[h, b]], ri[b, :rc[b]]), f"block {b}"
 
 
 def test_bs_all_blocks_equals_dense():
