@@ -58,7 +58,10 @@ __global__ void __launch_bounds__(320, PASS == 1 ? 2 : 1)
   using C = EstCfg<D, PASS>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
+  // heads vary fastest: the CTAs resident together take the same key tiles
+  // for every listed head, so that the heads of one KV group read each K tile
+  // from L2 after the first one brought it in
+  const int hi = blockIdx.x, chunk = blockIdx.y, b = blockIdx.z;
   const int head = p.heads[hi];
   if ((smem_u32(smem) & 1023u) != 0u || head < 0 || head >= p.Hq) {
     if (threadIdx.x == 0) report(p.status, MINF_ERR_DEVICE_BOUNDS, 60);
@@ -294,7 +297,7 @@ static cudaError_t launch_est_tc(const CUtensorMap& tq, const CUtensorMap& tk, c
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(vs_est_tc_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, C2::kSmem);
   if (e != cudaSuccess) return e;
-  const dim3 grid(nchunks, p.nh, p.B);
+  const dim3 grid(p.nh, nchunks, p.B);
   vs_est_tc_kernel<D, 1><<<grid, C1::kThreads, C1::kSmem, stream>>>(tq, tk, p, tpc, nchunks);
   e = vs_combine_launch(p, nchunks, stream);
   if (e != cudaSuccess) return e;
