@@ -202,8 +202,7 @@ def _barrier(dist):
 
 
 def _counters(ws):
-    c = ws[:24].cpu().view(torch.int64)
-    return int(c[1]), int(c[2])
+    return minf.attn_counters(ws)
 
 
 # ----------------------------------------------------------- CPU oracle leg

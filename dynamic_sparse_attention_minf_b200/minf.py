@@ -357,6 +357,13 @@ def minf_sparse_attn_layer(q, k, v, vs_heads=None, vs_index: VSIndex | None = No
     return o, lse
 
 
+def attn_counters(ws):
+    """(executed 128 x 128 key tiles, kept score entries) that the attention
+    launches on this workspace counted since it was zeroed."""
+    c = ws[:24].cpu().view(torch.int64)
+    return int(c[1]), int(c[2])
+
+
 def minf_get_device_status(ws, stream=None):
     return lib().minf_get_device_status(_p(ws), _stream(stream))
 

@@ -369,6 +369,24 @@ def attention_rows(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray,
     return o, lse
 
 
+def kept_mass(q_rows: np.ndarray, k: np.ndarray, rows: np.ndarray, mask: np.ndarray, scale: float):
+    """The share of each row's dense causal attention that a sparse mask keeps
+    (the quality measure of the offline pattern search, "MInference 1.0"
+    summary, "Summary", stage 1: a pattern per head chosen offline; the page
+    names no measure, and the kept probability mass is the plain reading):
+    for row i, the sum over j in M(i) of p_ij, p_ij = exp(s_ij) / sum_{j' <= i}
+    exp(s_ij'), s_ij = scale q_i . k_j.  Only the causal part of the mask
+    counts."""
+    q_rows = np.asarray(q_rows, np.float64)
+    rows = np.asarray(rows)
+    s = scale * (q_rows @ np.asarray(k, np.float64).T)
+    causal = np.arange(k.shape[0])[None, :] <= rows[:, None]
+    s = np.where(causal, s, NEG_INF)
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    return np.where(mask & causal, e, 0.0).sum(axis=1) / e.sum(axis=1)
+
+
 def attention_head(q, k, v, rows, mask_fn, scale, row_chunk: int = 0):
     """Attention of one head for the given query rows, in row chunks;
     ``mask_fn(rows)`` returns the boolean mask of those rows."""

@@ -200,6 +200,20 @@ def _attention_rows_variant(q_rows, k, v, mask, scale, *, lse_without_max=False,
     return o, lse
 
 
+def _kept_mass_variant(q_rows, k, rows, mask, scale, *, over_mask=False, noncausal=False):
+    q_rows = np.asarray(q_rows, np.float64)
+    rows = np.asarray(rows)
+    s = scale * (q_rows @ np.asarray(k, np.float64).T)
+    causal = np.arange(k.shape[0])[None, :] <= rows[:, None]
+    sc = np.where(causal, s, -np.inf)
+    e = np.exp(sc - sc.max(axis=1, keepdims=True))
+    keep = mask if noncausal else (mask & causal)
+    if noncausal:
+        e = np.exp(s - sc.max(axis=1, keepdims=True))
+    den = np.where(mask & causal, e, 0.0).sum(axis=1) if over_mask else np.where(causal, e, 0.0).sum(axis=1)
+    return np.where(keep, e, 0.0).sum(axis=1) / den
+
+
 def _to_f64_via_half(x):
     import torch
     if isinstance(x, torch.Tensor):
@@ -245,6 +259,10 @@ MUTANTS = {
     "default_scale: 1/d instead of 1/sqrt(d)": {"default_scale": lambda d: 1.0 / d},
     "kv_head: interleaved instead of contiguous groups": {"kv_head": lambda h, Hq, Hkv: h % Hkv},
     "to_f64: converted through float16": {"to_f64": _to_f64_via_half},
+    "kept_mass: normalised over the mask": {
+        "kept_mass": lambda q, k, r, m, sc: _kept_mass_variant(q, k, r, m, sc, over_mask=True)},
+    "kept_mass: keys past the row counted": {
+        "kept_mass": lambda q, k, r, m, sc: _kept_mass_variant(q, k, r, m, sc, noncausal=True)},
 }
 
 

@@ -468,3 +468,50 @@ def test_to_f64_is_exact_bf16_decoding():
         e, f = (b >> 7) & 0xFF, b & 0x7F
         ref = sign * (f / 128.0 * 2.0 ** -126 if e == 0 else (1 + f / 128.0) * 2.0 ** (e - 127))
         assert g == ref, (b, g, ref)
+
+
+# ---------------------------------------------------------- kept attention mass
+def test_kept_mass_bruteforce_loops_and_closed_forms():
+    """The kept share of a row's causal softmax, by plain loops; the full
+    causal mask keeps 1, the empty mask 0, a single key its probability, and
+    keys past the row do not count."""
+    rng = np.random.default_rng(5)
+    N, d = 24, 8
+    q = rng.normal(size=(N, d))
+    k = rng.normal(size=(N, d))
+    sc = 0.4
+    rows = np.array([0, 3, 11, 23])
+    mask = rng.random((rows.size, N)) < 0.4
+    got = orc.kept_mass(q[rows], k, rows, mask, sc)
+    for a, i in enumerate(rows):
+        w = [math.exp(sc * float(q[i] @ k[j])) for j in range(i + 1)]
+        kept = sum(w[j] for j in range(i + 1) if mask[a, j])
+        assert got[a] == pytest.approx(kept / sum(w), rel=1e-12, abs=1e-15)
+    full = np.ones((rows.size, N), bool)
+    np.testing.assert_allclose(orc.kept_mass(q[rows], k, rows, full, sc), 1.0, rtol=1e-12)
+    assert (orc.kept_mass(q[rows], k, rows, ~full, sc) == 0).all()
+    one = np.zeros((rows.size, N), bool)
+    one[:, 0] = True
+    p0 = [math.exp(sc * float(q[i] @ k[0])) / sum(math.exp(sc * float(q[i] @ k[j])) for j in range(i + 1))
+          for i in rows]
+    np.testing.assert_allclose(orc.kept_mass(q[rows], k, rows, one, sc), p0, rtol=1e-12)
+    past = np.zeros((rows.size, N), bool)
+    past[:, -1] = True  # key N-1 is past every row but the last
+    np.testing.assert_allclose(orc.kept_mass(q[rows], k, rows, past, sc)[:-1], 0.0)
+
+
+def test_kept_mass_equals_lse_ratio():
+    """For a causal mask M, the kept mass of row i is exp(LSE over M minus the
+    dense causal LSE): the identity the pattern search reads off the kernels'
+    LSE outputs."""
+    rng = np.random.default_rng(6)
+    N, d = 40, 16
+    q, k, v = rng.normal(size=(N, d)), rng.normal(size=(N, d)), rng.normal(size=(N, d))
+    sc = 0.25
+    rows = np.arange(N)
+    causal = np.arange(N)[None, :] <= rows[:, None]
+    mask = (rng.random((N, N)) < 0.5) & causal
+    mask[rows, rows] = True  # every row keeps at least its diagonal
+    _, lse_s = orc.attention_rows(q, k, v, mask, sc)
+    _, lse_d = orc.attention_rows(q, k, v, causal, sc)
+    np.testing.assert_allclose(orc.kept_mass(q, k, rows, mask, sc), np.exp(lse_s - lse_d), rtol=1e-12)
