@@ -202,6 +202,7 @@ def _barrier(dist):
 
 
 def _counters(ws):
+    from dynamic_sparse_attention_minf_b200 import minf
     return minf.attn_counters(ws)
 
 
@@ -544,7 +545,9 @@ def run_kernel_case(args):
     """One kernel on a small case, for profilers: ``--kernel dense|vs`` at
     ``--N`` tokens (8 query / 2 KV heads, d = 128; the VS case uses the 1M
     workload's budgets, vertical 2000 / slash 12000).  The index is built
-    once; then the kernel runs ``--warmup`` + ``--steps`` times."""
+    once; then the kernel runs ``--warmup`` + ``--steps`` times.
+    ``--kernel vs_est|bs_est`` runs the index estimation of those 8 heads
+    instead (vertical 2000 / slash 12000; top-100 blocks)."""
     from dynamic_sparse_attention_minf_b200 import layer, minf
     from dynamic_sparse_attention_minf_b200 import workloads as wl
     w = wl.config(WORKLOAD_ID, N=args.N)
@@ -552,6 +555,21 @@ def run_kernel_case(args):
     w.patterns = [wl.PAT_VS] * 8
     q, k, v = wl.make_qkv(w, "cuda")
     o = torch.empty_like(q)
+    if args.kernel in ("vs_est", "bs_est"):
+        shp = minf.shape_of(q, k)
+        heads = list(range(8))
+        if args.kernel == "vs_est":
+            ws = minf.workspace(minf.OP_ESTIMATE_VS, shp, 8)
+            fn = lambda: minf.minf_estimate_vs(q, k, heads, w.k_v, w.k_s, ws=ws)
+        else:
+            ws = minf.workspace(minf.OP_ESTIMATE_BS, shp, 8, k_b=100)
+            fn = lambda: minf.minf_estimate_bs(q, k, heads, 100, ws=ws)
+        for _ in range(args.warmup + args.steps):
+            fn()
+        torch.cuda.synchronize()
+        print(json.dumps({"kernel": args.kernel, "N": args.N, "launches": args.warmup + args.steps,
+                          "status": minf.minf_get_device_status(ws)}))
+        return
     if args.kernel == "vs":
         plan = layer.make_plan(w, "cuda")
         layer.run_layer(plan, q, k, v, o)
@@ -586,7 +604,7 @@ def main():
     ap.add_argument("--config", type=int, default=WORKLOAD_ID, choices=[2, 3, 4],
                     help="workload: 4 (default) the 1M-token mixed layer, 2 the 128K mixed layer, "
                          "3 the 512K all-Vertical-Slash layer")
-    ap.add_argument("--kernel", choices=["dense", "vs"], default=None,
+    ap.add_argument("--kernel", choices=["dense", "vs", "vs_est", "bs_est"], default=None,
                     help="run only this attention kernel on a small case (for profiling)")
     ap.add_argument("--N", type=int, default=262144, help="tokens of the --kernel case")
     ap.add_argument("--shard", choices=["kv", "replicas"], default="kv",

@@ -349,13 +349,20 @@ __device__ uint32_t tk_compact(uint32_t* keys, int32_t* cols, int n, int k, int 
   return T;
 }
 
+__device__ __forceinline__ float tk_key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
+}
+
 // One warp per query block b: the k best key blocks c <= b of its score row
 // (b itself forced), written ascending and padded with -1.  Rows are taken
-// longest first; each chunk's loads are issued while the chunk before is
-// filtered.
+// longest first.  Lane l holds the four consecutive columns hi - 4l - u,
+// u = 0..3, of a 128-column chunk, so that lane-major order is descending
+// column order; a chunk's loads are issued while the chunk before is
+// filtered.  Columns are compared with the threshold as floats (the order
+// keys order them alike); only the survivors get their keys.
 __global__ void __launch_bounds__(32 * kTkWarps, 4) bs_topk_warp_kernel(const float* __restrict__ scores, int nb,
-                                                                    int bh_total, int k, int32_t* blk_idx,
-                                                                    int32_t* blk_cnt) {
+                                                                       int bh_total, int k, int32_t* blk_idx,
+                                                                       int32_t* blk_cnt) {
   __shared__ uint32_t skeys[kTkWarps][kTkCap];
   __shared__ int32_t scols[kTkWarps][kTkCap];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -367,47 +374,63 @@ __global__ void __launch_bounds__(32 * kTkWarps, 4) bs_topk_warp_kernel(const fl
   const float* sr = scores + row * nb;
   uint32_t* keys = skeys[warp];
   int32_t* cols = scols[warp];
-  const uint32_t lt = (1u << lane) - 1u;
-  // column hi - 32 u - lane of a chunk: descending in (u, lane)
   auto load = [&](int hi, float (&v)[4]) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int c = hi - 32 * u - lane;
+      const int c = hi - 4 * lane - u;
       v[u] = (c >= 0) ? __ldg(sr + c) : 0.f;
     }
   };
   int cnt = 0;
   bool have = false;  // a threshold exists once the list was compacted
   uint32_t tau = 0;
+  float tauf = 0.f;
   float cur[4];
   load(b, cur);
   for (int hi = b; hi >= 0; hi -= kTkChunk) {
     float nxt[4];
     if (hi - kTkChunk >= 0) load(hi - kTkChunk, nxt);
-    uint32_t key[4];
-    uint32_t s = 0;
+    // survivors: valid columns at or above the threshold (a value equal to
+    // it has a lower column than the list's entries of that key, so it ranks
+    // above them), and the forced diagonal
+    auto survivors = [&]() {
+      uint32_t m = 0;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = hi - 32 * u - lane;
-      key[u] = (c < 0) ? 0u : (c == b) ? 0xFFFFFFFFu : sel_order_key(cur[u]);
-      s += (key[u] != 0u && (!have || key[u] >= tau));
-    }
-    if (cnt + (int)__reduce_add_sync(0xFFFFFFFFu, s) > kTkCap) {
+      for (int u = 0; u < 4; ++u) {
+        const int c = hi - 4 * lane - u;
+        m |= (uint32_t)(c >= 0 && (!have || cur[u] >= tauf || c == b)) << u;
+      }
+      return m;
+    };
+    uint32_t m = survivors();
+    int tot = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)__popc(m));
+    if (cnt + tot > kTkCap) {
       tau = tk_compact(keys, cols, cnt, k, lane);
+      tauf = tk_key_value(tau);
       cnt = k;
       have = true;
+      m = survivors();
+      tot = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)__popc(m));
     }
-    // a key equal to the threshold has a lower column than the list's
-    // entries of that key, so it ranks above them and is kept too
+    if (tot) {
+      const int n = __popc(m);
+      int incl = n;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const bool keep = key[u] != 0u && (!have || key[u] >= tau);
-      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
-      if (keep) {
-        keys[cnt + __popc(bal & lt)] = key[u];
-        cols[cnt + __popc(bal & lt)] = hi - 32 * u - lane;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
       }
-      cnt += __popc(bal);
+      int pos = cnt + incl - n;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if ((m >> u) & 1u) {
+          const int c = hi - 4 * lane - u;
+          keys[pos] = (c == b) ? 0xFFFFFFFFu : sel_order_key(cur[u]);
+          cols[pos] = c;
+          ++pos;
+        }
+      }
+      cnt += tot;
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) cur[u] = nxt[u];

@@ -54,3 +54,12 @@ def test_recorded_traffic_gated_by_digest(monkeypatch):
     assert t is None or t > 0
     monkeypatch.setattr(bench, "kernel_sources_digest", lambda: "0" * 64)
     assert bench._recorded_traffic() is None
+
+
+def test_attention_counters_read_from_a_workspace():
+    """The bench's tile and kept-entry counters come from the status block of
+    an attention workspace (bytes 8..23)."""
+    import torch
+    ws = torch.zeros(256, dtype=torch.uint8)
+    ws[8:24].view(torch.int64)[:] = torch.tensor([12345, 678])
+    assert bench._counters(ws) == (12345, 678)
