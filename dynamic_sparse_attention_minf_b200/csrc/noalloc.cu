@@ -13,15 +13,14 @@
 // The array is a file-scope device variable of kNoAllocScratchBytes, so every
 // GPU on which the library's module is loaded keeps it for the life of the
 // process.  In host code its name is only a host-side stand-in for the device
-// variable; the device address is fetched once per device with
-// cudaGetSymbolAddress (while that device is current) and cached.  The first
-// call on a device performs that set-up, so it should be made before any
-// stream capture starts.  All calls share the array and it keeps the last
-// call's contents: the status word at its head is cleared on every call, the
-// rest is fully rewritten before it is read.  Calls whose executions overlap
-// on the GPU (different streams, or different host threads) race on the
-// array; serialise them.
-#include <mutex>
+// variable; every call fetches the device address with cudaGetSymbolAddress
+// (while the device is current), which allocates nothing.  The first call on
+// a device loads the module, so it should be made before any stream capture
+// starts.  All calls share the array and it keeps the last call's contents:
+// the status word at its head is cleared on every call (and by
+// minf_noalloc_device_status, which reads it), the rest is fully rewritten
+// before it is read.  Calls whose executions overlap on the GPU (different
+// streams, or different host threads) race on the array; serialise them.
 
 #include "minf_device.cuh"
 #include "minf_internal.h"
@@ -29,24 +28,16 @@
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = 64ull << 20;  // 64 MiB
-constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_vs_scratch[kNoAllocScratchBytes];
 
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_vs_scratch on the current device (looked up once).
+// Device address of g_vs_scratch on the current device.  Looked up on every
+// call (a lookup allocates nothing), so that the address follows a reloaded
+// module after cudaDeviceReset.
 minf_status scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MINF_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_vs_scratch) != cudaSuccess || p == nullptr) return MINF_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_vs_scratch) != cudaSuccess || p == nullptr) return MINF_ERR_CUDA;
+  *out = p;
   return MINF_OK;
 }
 
@@ -65,4 +56,15 @@ extern "C" minf_status minf_estimate_vs_noalloc(const minf_shape* shape, const m
   if (cudaMemsetAsync(scratch, 0, 256, (cudaStream_t)stream) != cudaSuccess) return MINF_ERR_CUDA;
   return minf_estimate_vs(shape, Q, K, heads, nh, last_q, k_v, k_s, v_idx, s_idx, v_score, s_score, scratch,
                           kNoAllocScratchBytes, stream);
+}
+
+extern "C" minf_status minf_noalloc_device_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MINF_ERR_CUDA;
+  int code = 0;  // the status block's first word: the first error code recorded
+  if (cudaMemcpyFromSymbol(&code, g_vs_scratch, sizeof(code), 0, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MINF_ERR_CUDA;
+  const int zero[2] = {0, 0};  // code and site
+  if (code != 0 && cudaMemcpyToSymbol(g_vs_scratch, zero, sizeof(zero), 0, cudaMemcpyHostToDevice) != cudaSuccess)
+    return MINF_ERR_CUDA;
+  return (minf_status)code;
 }

@@ -391,6 +391,15 @@ def minf_estimate_vs_noalloc(q, k, heads, k_v, k_s, last_q=64, scale=0.0, return
     return (v_idx, s_idx, vs, ss) if return_scores else (v_idx, s_idx)
 
 
+def minf_noalloc_device_status(stream=None):
+    """The status word of minf_estimate_vs_noalloc's built-in scratch
+    (synchronizes the stream; reading clears it)."""
+    fn = lib().minf_noalloc_device_status
+    fn.argtypes = [ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    return int(fn(_stream(stream)))
+
+
 def minf_selftest_exp2(x, stream=None):
     """The softmax's two exponentials on device floats x: (polynomial, MUFU)."""
     x = x.contiguous().float()

@@ -163,15 +163,25 @@ minf_status minf_estimate_vs(const minf_shape* shape, const minf_bf16* Q, const 
  * exits.  Problems that need more scratch than that (minf_workspace_size for
  * MINF_OP_ESTIMATE_VS above 64 MiB, about 3.5M (batch x heads x tokens))
  * are rejected with MINF_ERR_WORKSPACE_TOO_SMALL before anything runs.  The
- * call allocates nothing.  Its first call on a device looks up the array's
- * device address, so make that call before any stream capture begins.  All
- * calls share the one array: calls that overlap on the GPU race, so
- * serialise them.  This variant has no readable device status word.
+ * call allocates nothing.  Every call looks up the array's device address
+ * (which follows a module reloaded after cudaDeviceReset); the first call on
+ * a device loads the library's device code, so make it before any stream
+ * capture begins.  All calls share the one array: calls that overlap on the
+ * GPU race, so serialise them.  Device-side errors are latched in the
+ * array's status word: read them with minf_noalloc_device_status.
  */
 minf_status minf_estimate_vs_noalloc(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K,
                                      const int32_t* heads, int nh, int last_q, int k_v, int k_s,
                                      int32_t* v_idx, int32_t* s_idx, float* v_score, float* s_score,
                                      void* stream);
+
+/*
+ * Synchronizes `stream` and returns the device status word of the built-in
+ * scratch array of minf_estimate_vs_noalloc (MINF_OK when no kernel reported
+ * an error since the last read), then clears it.  Copies to and from host
+ * memory only: it allocates nothing.  Not for use during a stream capture.
+ */
+minf_status minf_noalloc_device_status(void* stream);
 
 /*
  * Block-Sparse index estimation (summary, "Key points": queries and keys are

@@ -75,3 +75,66 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     big = minf.Shape(1, 32, 8, 1048576, 128, 0.0)    # 32 heads x 1M tokens: far above 64 MiB
     fake = ctypes.c_void_p(1 << 20)
     assert fn(ctypes.byref(big), fake, fake, fake, 32, 64, 8, 8, fake, fake, None, None, None) == 4
+
+
+def test_noalloc_reports_a_bad_head_through_its_status_getter():
+    """A head id outside [0, Hq) is reported by the estimation kernels into
+    the built-in scratch's status word; the getter returns it once and clears
+    it, and a good call afterwards leaves it clear."""
+    w = wl.small(Hq=4, Hkv=2, N=1024, d=128, seed=33, k_v=32, k_s=64)
+    q, k, _ = wl.make_qkv(w, "cuda")
+    assert minf.minf_noalloc_device_status() == 0
+    minf.minf_estimate_vs_noalloc(q, k, [1, 99], w.k_v, w.k_s)
+    assert minf.minf_noalloc_device_status() == 6   # MINF_ERR_DEVICE_BOUNDS
+    assert minf.minf_noalloc_device_status() == 0
+    got = minf.minf_estimate_vs_noalloc(q, k, [1, 2], w.k_v, w.k_s)
+    ref = minf.minf_estimate_vs(q, k, [1, 2], w.k_v, w.k_s)
+    assert minf.minf_noalloc_device_status() == 0
+    assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1])
+
+
+def test_noalloc_captures_in_a_graph_without_allocating():
+    """The reason the entry point exists: captured into a CUDA graph under the
+    global capture mode (where an allocating call would invalidate the
+    capture) and replayed, it gives the workspace path's indices, and neither
+    torch's allocator nor the device's free memory moves against it."""
+    w = wl.small(Hq=4, Hkv=2, N=2048, d=128, seed=35, k_v=64, k_s=128)
+    q, k, _ = wl.make_qkv(w, "cuda")
+    heads = [0, 3]
+    hd = torch.tensor(heads, dtype=torch.int32, device="cuda")
+    ref = minf.minf_estimate_vs(q, k, heads, w.k_v, w.k_s)
+    L = minf.lib()
+    fn = L.minf_estimate_vs_noalloc
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(minf.Shape), vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    shp = minf.shape_of(q, k)
+    v_idx = torch.full((1, 2, w.k_v), -7, dtype=torch.int32, device="cuda")
+    s_idx = torch.full((1, 2, w.k_s), -7, dtype=torch.int32, device="cuda")
+    args = lambda st: (ctypes.byref(shp), vp(q.data_ptr()), vp(k.data_ptr()), vp(hd.data_ptr()), 2, 64,
+                       w.k_v, w.k_s, vp(v_idx.data_ptr()), vp(s_idx.data_ptr()), None, None, vp(st))
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        assert fn(*args(side.cuda_stream)) == 0      # warm-up outside the capture
+    torch.cuda.synchronize()
+    alloc0 = torch.cuda.memory_allocated()
+    g = torch.cuda.CUDAGraph()
+    codes = []
+    # an allocating call inside the capture would invalidate it (global mode)
+    with torch.cuda.graph(g, stream=side, capture_error_mode="global"):
+        codes.append(fn(*args(side.cuda_stream)))
+    assert codes == [0]
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()   # after the graph is instantiated
+    for _ in range(2):
+        v_idx.fill_(-7)
+        s_idx.fill_(-7)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(v_idx, ref[0]) and torch.equal(s_idx, ref[1])
+    assert minf.minf_noalloc_device_status() == 0
+    # nothing was allocated: neither torch's allocator nor the device grew
+    assert torch.cuda.memory_allocated() <= alloc0
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 >= free0
+    del g
