@@ -18,8 +18,9 @@
 //          shared memory, and the CTA forms, in a fixed order, the column
 //          sums (vertical scores) and the tile's 191 diagonal partials.
 //
-// warps 0-7: score warps; warp 8 lane 0: TMA producer; warp 9: TMEM owner and
-// MMA issuer.
+// Score warps: 8 (pass 1) or 16 (pass 2: two groups of 8 on alternate key
+// tiles, each with its own P buffer); then one warp whose lane 0 is the TMA
+// producer, and one TMEM-owning MMA issuer warp.
 #include <algorithm>
 
 #include "minf_device.cuh"
@@ -29,10 +30,14 @@ namespace minf {
 
 // Pass 1 needs no P buffer: two K stages keep its CTA under half of an SM's
 // shared memory, so that two CTAs share each SM and hide each other's waits.
+// Pass 2 runs two groups of eight score warps, on the even and the odd key
+// tiles, so that one group's shared-memory sums overlap the other's scores.
 template <int D, int PASS>
 struct EstCfg {
-  static constexpr int kThreads = 320;
-  static constexpr int kScoreThreads = 256;
+  static constexpr int kGroups = (PASS == 1) ? 1 : 2;
+  static constexpr int kScoreWarps = 8 * kGroups;
+  static constexpr int kThreads = 32 * (kScoreWarps + 2);
+  static constexpr int kScoreThreads = 256;  // per group
   static constexpr int kRegion = 128 * 128;
   static constexpr int kTileBytes = 128 * D * 2;  // 128 rows (Q twice) or 128 keys (K)
   static constexpr int kStages = (PASS == 1) ? 2 : 3;
@@ -52,7 +57,7 @@ struct EstCfg {
 };
 
 template <int D, int PASS>
-__global__ void __launch_bounds__(320, PASS == 1 ? 2 : 1)
+__global__ void __launch_bounds__(EstCfg<D, PASS>::kThreads, PASS == 1 ? 2 : 1)
     vs_est_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const VsEstParams p, int tiles_per_cta, int nchunks) {
   using C = EstCfg<D, PASS>;
@@ -97,7 +102,8 @@ __global__ void __launch_bounds__(320, PASS == 1 ? 2 : 1)
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  const int w_prod = C::kScoreWarps, w_mma = C::kScoreWarps + 1;
+  if (warp == w_mma) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
@@ -106,7 +112,7 @@ __global__ void __launch_bounds__(320, PASS == 1 ? 2 : 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == w_prod) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       // Q's last 64 rows into rows 0-63 and again into rows 64-127
@@ -137,7 +143,7 @@ __global__ void __launch_bounds__(320, PASS == 1 ? 2 : 1)
         mbar_wait(&k_full[k % C::kStages], (k / C::kStages) & 1, &dummy, p.status, 62);
       mbar_wait(q_full, 0, &dummy, p.status, 63);
     }
-  } else if (warp == 9) {
+  } else if (warp == w_mma) {
     // --------------------------------------------------------- MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(q_full, 0, abort, p.status, 64);
@@ -165,8 +171,11 @@ __global__ void __launch_bounds__(320, PASS == 1 ? 2 : 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------- score warps
-    const int qq = warp & 3;                      // TMEM lane quarter
-    const int grp = (qq >> 1) * 2 + (warp >> 2);  // column group: key columns 32 grp .. 32 grp + 31
+    const int sg = warp >> 3;                     // warp group: key tiles sg, sg + kGroups, ...
+    const int ww = warp & 7;
+    const int qq = ww & 3;                        // TMEM lane quarter (warp & 3)
+    const int grp = (qq >> 1) * 2 + (ww >> 2);    // column group: key columns 32 grp .. 32 grp + 31
+    const int bar_sync = 1 + 2 * sg, bar_vote = 2 + 2 * sg;  // this group's named barriers
     const int qrow = (qq & 1) * 32 + lane;        // query row N - 64 + qrow
     const int i = p.N - 64 + qrow;
     const bool real = qrow >= 64 - p.last_q;
@@ -178,12 +187,12 @@ __global__ void __launch_bounds__(320, PASS == 1 ? 2 : 1)
       mr = p.row_ml[(bh * 64 + qrow) * 2];
       il = p.row_ml[(bh * 64 + qrow) * 2 + 1];
     }
-    for (int k = 0; k < nt; ++k) {
+    for (int k = sg; k < nt; k += C::kGroups) {
       const int buf = k & 1;
-      // all score warps agree before going on (pass 2 meets at a barrier
-      // below, which a warp that gave up would never reach)
+      // all score warps of the group agree before going on (pass 2 meets at a
+      // barrier below, which a warp that gave up would never reach)
       const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (k >> 1) & 1, abort, p.status, 68));
-      if (!bar_and(2, C::kScoreThreads, got)) break;
+      if (!bar_and(bar_vote, C::kScoreThreads, got)) break;
       tc_fence_after();
       uint32_t v0[32];
       tmem_ld32(taddr + buf * 128, v0);
@@ -217,8 +226,8 @@ __global__ void __launch_bounds__(320, PASS == 1 ? 2 : 1)
 #pragma unroll
         for (int c = 0; c < 32; ++c)
           P[qrow * C::kPStride + grp * 32 + c] = (x[c] == -INFINITY) ? 0.f : fast_exp2(x[c] - mr) * il;
-        named_bar_sync(1, C::kScoreThreads);
-        const int tid = threadIdx.x;  // 0 .. 255
+        named_bar_sync(bar_sync, C::kScoreThreads);
+        const int tid = threadIdx.x & 255;  // 0 .. 255 within the group
         // Fixed-order sums over the tile's 64 rows, each as four interleaved
         // partial sums (rows q = 0, 1, 2, 3 mod 4) added in a fixed order.
         // Threads 0-127: vertical score of key column tid, then (0-62) the
@@ -256,7 +265,7 @@ __global__ void __launch_bounds__(320, PASS == 1 ? 2 : 1)
       float* xch = reinterpret_cast<float*>(smem + C::kOffXch);
       xch[(grp * 64 + qrow) * 2] = m;
       xch[(grp * 64 + qrow) * 2 + 1] = l;
-      named_bar_sync(1, C::kScoreThreads);
+      named_bar_sync(bar_sync, C::kScoreThreads);
       if (grp == 0) {
         float M = -INFINITY;
 #pragma unroll
@@ -277,7 +286,7 @@ __global__ void __launch_bounds__(320, PASS == 1 ? 2 : 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == w_mma) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
