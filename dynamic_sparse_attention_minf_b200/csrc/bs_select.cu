@@ -359,7 +359,9 @@ __device__ __forceinline__ float tk_key_value(uint32_t key) {
 // u = 0..3, of a 128-column chunk, so that lane-major order is descending
 // column order; a chunk's loads are issued while the chunk before is
 // filtered.  Columns are compared with the threshold as floats (the order
-// keys order them alike); only the survivors get their keys.
+// keys order them alike; the threshold is -inf until the first compaction,
+// columns before 0 load as NaN, which no comparison keeps, and the forced
+// diagonal loads as +inf); only the survivors get their keys.
 __global__ void __launch_bounds__(32 * kTkWarps, 4) bs_topk_warp_kernel(const float* __restrict__ scores, int nb,
                                                                        int bh_total, int k, int32_t* blk_idx,
                                                                        int32_t* blk_cnt) {
@@ -378,37 +380,31 @@ __global__ void __launch_bounds__(32 * kTkWarps, 4) bs_topk_warp_kernel(const fl
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int c = hi - 4 * lane - u;
-      v[u] = (c >= 0) ? __ldg(sr + c) : 0.f;
+      v[u] = (c >= 0) ? __ldg(sr + c) : __int_as_float(0x7FC00000);  // NaN
     }
   };
   int cnt = 0;
-  bool have = false;  // a threshold exists once the list was compacted
-  uint32_t tau = 0;
-  float tauf = 0.f;
+  float tauf = -INFINITY;  // the threshold as a value: -inf until the first compaction
   float cur[4];
   load(b, cur);
+  if (lane == 0) cur[0] = INFINITY;  // column b: the forced diagonal
   for (int hi = b; hi >= 0; hi -= kTkChunk) {
     float nxt[4];
     if (hi - kTkChunk >= 0) load(hi - kTkChunk, nxt);
-    // survivors: valid columns at or above the threshold (a value equal to
-    // it has a lower column than the list's entries of that key, so it ranks
-    // above them), and the forced diagonal
+    // survivors: columns at or above the threshold (a value equal to it has
+    // a lower column than the list's entries of that key, so it ranks above
+    // them)
     auto survivors = [&]() {
       uint32_t m = 0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = hi - 4 * lane - u;
-        m |= (uint32_t)(c >= 0 && (!have || cur[u] >= tauf || c == b)) << u;
-      }
+      for (int u = 0; u < 4; ++u) m |= (uint32_t)(cur[u] >= tauf) << u;
       return m;
     };
     uint32_t m = survivors();
     int tot = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)__popc(m));
     if (cnt + tot > kTkCap) {
-      tau = tk_compact(keys, cols, cnt, k, lane);
-      tauf = tk_key_value(tau);
+      tauf = tk_key_value(tk_compact(keys, cols, cnt, k, lane));
       cnt = k;
-      have = true;
       m = survivors();
       tot = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)__popc(m));
     }
