@@ -612,7 +612,12 @@ cudaError_t topk_rows_launch(const TopkRows& t, cudaStream_t stream) {
 
 // ====================================================== Block-Sparse scores
 // Mean of every 64-row block of Q (listed heads) and K (their KV heads), fp32.
-__global__ void bs_pool_kernel(const BsEstParams p) {
+// One CTA of 256 threads per (64-row block, head slot): threads 0-127 pool Q,
+// 128-255 K.  Within a matrix a thread sums 8 adjacent columns (16-byte
+// loads) over every (128 / (d / 8))-th row of the block; the row phases are
+// then added in a fixed order, one thread per column.
+__global__ void __launch_bounds__(256) bs_pool_kernel(const BsEstParams p) {
+  __shared__ float red[2][16][128];  // [matrix][row phase][column]
   const int qb = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
   const int head = p.heads[hi];
   if (head < 0 || head >= p.Hq) {
@@ -621,12 +626,32 @@ __global__ void bs_pool_kernel(const BsEstParams p) {
   }
   const int nb = p.N / 64;
   const int kvh = head / p.group;
-  const int dd = threadIdx.x % p.d;
-  const bool isk = threadIdx.x >= p.d;
-  const __nv_bfloat16* src = isk ? p.K + ((size_t)(b * p.Hkv + kvh) * p.N + qb * 64) * p.d
-                                 : p.Q + ((size_t)(b * p.Hq + head) * p.N + qb * 64) * p.d;
+  const int nc = p.d / 8;     // 16-byte column groups of a row
+  const int per = 128 / nc;   // row phases
+  {
+    const int isk = threadIdx.x >> 7, t = threadIdx.x & 127;
+    const int cg = t % nc, rp = t / nc;
+    const __nv_bfloat16* src = isk ? p.K + ((size_t)(b * p.Hkv + kvh) * p.N + qb * 64) * p.d
+                                   : p.Q + ((size_t)(b * p.Hq + head) * p.N + qb * 64) * p.d;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int r = rp; r < 64; r += per) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * p.d + 8 * cg));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += __uint_as_float(w[e] << 16);
+        acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[isk][rp][8 * cg + e] = acc[e];
+  }
+  __syncthreads();
+  if (threadIdx.x >= 2 * p.d) return;
+  const int isk = threadIdx.x / p.d, dd = threadIdx.x % p.d;
   float s = 0.f;
-  for (int r = 0; r < 64; ++r) s += __bfloat162float(src[(size_t)r * p.d + dd]);
+  for (int rp = 0; rp < per; ++rp) s += red[isk][rp][dd];
   const size_t at = (((size_t)(b * p.nh + hi) * nb) + qb) * p.d + dd;
   const float m = s * (1.0f / 64.0f);
   (isk ? p.kbar : p.qbar)[at] = m;
@@ -774,7 +799,7 @@ __global__ void __launch_bounds__(256) bs_score_tri_kernel(const BsEstParams p, 
 
 cudaError_t bs_pool_score_launch(const BsEstParams& p, cudaStream_t stream) {
   const int nb = p.N / 64;
-  bs_pool_kernel<<<dim3(nb, p.nh, p.B), 2 * p.d, 0, stream>>>(p);
+  bs_pool_kernel<<<dim3(nb, p.nh, p.B), 256, 0, stream>>>(p);
   if (!p.scores) return cudaGetLastError();
   if (nb % 8 == 0 && p.d % kBsK == 0) {
     const int nt = (nb + kBsT - 1) / kBsT;
