@@ -154,44 +154,59 @@ __global__ void __launch_bounds__(256) vs_vlist_kernel(const VsIndexParams p, co
 }
 
 // One warp per 128-row query tile t (blocks b0 = 2t, b1 = 2t + 1, first row
-// R): the columns the tile gathers, with the blocks whose lists hold them.
+// R): the vertical lists of both blocks and the columns the tile gathers.
 // Column j is listed for block b (first row r0) when j <= r0 + 63 and bit
-// (r0 - j + 63) of the group bitmap is clear.  Entries: first every column of
-// block b1's list (bit 31; bit 30 too if block b0 lists it), then the columns
-// of block b0's list that block b1 does not list (bit 30 only).
-__global__ void __launch_bounds__(256) vs_tlist_kernel(const VsIndexParams p, int32_t* tvcnt, int32_t* tvidx) {
+// (r0 - j + 63) of the group bitmap is clear.  The tile's entries: first every
+// column of block b1's list (bit 31; bit 30 too if block b0 lists it), then
+// the columns of block b0's list that block b1 does not list (bit 30 only).
+// The first pass over the ascending verticals writes both block lists and the
+// first part; a second, up to row R + 63, the second part after it.
+__global__ void __launch_bounds__(256) vs_tile_lists_kernel(const VsIndexParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nt = p.N / 128;
+  const int nt = p.N / 128, nb = p.N / 64;
   const int qt = blockIdx.x * 8 + warp;
   const int hi = blockIdx.y, b = blockIdx.z;
   if (qt >= nt) return;
   const size_t bh = (size_t)b * p.nh + hi;
   const int* v = p.v_idx + bh * p.k_v;
   const uint32_t* W = p.idx.wmap + bh * p.wmap_words;
-  int32_t* out = tvidx + (bh * nt + qt) * (size_t)p.k_v;
+  int32_t* out = p.idx.tvidx + (bh * nt + qt) * (size_t)p.k_v;
+  int32_t* list0 = p.idx.vidx + (bh * nb + 2 * qt) * (size_t)p.k_v;
+  int32_t* list1 = list0 + p.k_v;
   const int R = qt * 128;
+  const uint32_t lt = (1u << lane) - 1u;
   auto covered = [&](int bit) -> bool { return (__ldg(W + (bit >> 5)) >> (bit & 31)) & 1u; };
-  int n = 0;
+  int n = 0, n0 = 0;
   for (int pass = 0; pass < 2; ++pass) {
+    const int last = R + (pass == 0 ? 127 : 63);
     for (int base = 0; base < p.k_v; base += 32) {
       const int x = base + lane;
       const int j = (x < p.k_v) ? v[x] : 0x7FFFFFFF;
-      const bool inr = (j >= 0) && (j <= R + 127);
-      bool keep = false;
-      uint32_t e = 0;
+      const bool inr = (j >= 0) && (j <= last);
+      bool in0 = false, in1 = false;
       if (inr) {
-        const bool in0 = (j <= R + 63) && !covered(R - j + 63);  // block b0 lists j
-        const bool in1 = !covered(R + 127 - j);                   // block b1 lists j
-        keep = (pass == 0) ? in1 : (in0 && !in1);
-        e = (uint32_t)j | (in0 ? (1u << 30) : 0u) | (in1 ? (1u << 31) : 0u);
+        in0 = (j <= R + 63) && !covered(R - j + 63);  // block b0 lists j
+        in1 = !covered(R + 127 - j);                   // block b1 lists j
       }
+      const bool keep = (pass == 0) ? in1 : (in0 && !in1);
+      const uint32_t e = (uint32_t)j | (in0 ? (1u << 30) : 0u) | (in1 ? (1u << 31) : 0u);
       const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
-      if (keep) out[n + __popc(bal & ((1u << lane) - 1u))] = (int32_t)e;
+      if (keep) out[n + __popc(bal & lt)] = (int32_t)e;
       n += __popc(bal);
+      if (pass == 0) {
+        const uint32_t b0 = __ballot_sync(0xFFFFFFFFu, in0);
+        if (in0) list0[n0 + __popc(b0 & lt)] = j;
+        if (in1) list1[__popc(bal & lt) + (n - __popc(bal))] = j;
+        n0 += __popc(b0);
+      }
       if (!__all_sync(0xFFFFFFFFu, inr || x >= p.k_v)) break;  // list is ascending
     }
+    if (pass == 0 && lane == 0) {
+      p.idx.vcnt[bh * nb + 2 * qt] = n0;
+      p.idx.vcnt[bh * nb + 2 * qt + 1] = n;
+    }
   }
-  if (lane == 0) tvcnt[bh * nt + qt] = n;
+  if (lane == 0) p.idx.tvcnt[bh * nt + qt] = n;
 }
 
 // One thread per word of the offset and key bitmaps: bit o of sbits set iff
@@ -220,11 +235,8 @@ cudaError_t vs_index_launch(const VsIndexParams& p, cudaStream_t stream) {
   vs_groups_kernel<<<dim3(p.nh, p.B), 1024, 0, stream>>>(p);
   vs_wmap_kernel<64><<<dim3((p.wmap_words + 255) / 256, p.nh, p.B), 256, 0, stream>>>(
       p, p.idx.grp, p.idx.grp_cnt, p.idx.wmap, p.wmap_words);
-  const int nb = p.N / 64;
-  vs_vlist_kernel<64><<<dim3((nb + 7) / 8, p.nh, p.B), 256, 0, stream>>>(p, p.idx.wmap, p.wmap_words, p.idx.vcnt,
-                                                                        p.idx.vidx);
   const int nt = p.N / 128;
-  vs_tlist_kernel<<<dim3((nt + 7) / 8, p.nh, p.B), 256, 0, stream>>>(p, p.idx.tvcnt, p.idx.tvidx);
+  vs_tile_lists_kernel<<<dim3((nt + 7) / 8, p.nh, p.B), 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -90,13 +90,13 @@ TOPK_LONG_ROW = 32768
 
 def launches_per_step(plan: LayerPlan, fused: bool = True) -> int:
     """Kernels one run_layer call launches: VS estimation (two score passes,
-    row combine, slash combine, two top-k), VS index build 4, BS estimation
+    row combine, slash combine, two top-k), VS index build 3, BS estimation
     3 (pool, pooled scores, top-k), and the attention: one launch for every
     head (fused) or one per pattern."""
     n = 0
     if plan.vs_heads is not None:
         topk = 9 if plan.w.N > TOPK_LONG_ROW else 1
-        n += 4 + 2 * topk + 4
+        n += 4 + 2 * topk + 3
     if plan.bs_heads is not None:
         n += 3
     if fused:

@@ -27,19 +27,19 @@ def test_launches_per_step_matches_launch_list_profile():
     m = re.search(r"(\d+) launches of libminf kernels in all = (\d+) x (\d+) \+ (\d+) x (\d+)", text)
     total, lf, nf, ls, ns = (int(g) for g in m.groups())
     listed = sum(int(c) for c in re.findall(r"^\| `minf::[^|]*\| (\d+) \|", text, re.M))
-    assert (nf, ns) == (n, n_sep) == (30, 32)
+    assert (nf, ns) == (n, n_sep) == (29, 31)
     assert listed == total == lf * nf + ls * ns
     attn = sum(int(c) for c in re.findall(r"^\| `minf::attn_kernel[^|]*\| (\d+) \|", text, re.M))
     assert attn == lf + 3 * ls
 
 
 def test_launches_per_step_other_layers():
-    # 512K, Vertical-Slash heads only: estimation 4 + two 9-launch top-k, index 4, attention 1
-    assert layer.launches_per_step(_plan(3)) == 27
+    # 512K, Vertical-Slash heads only: estimation 4 + two 9-launch top-k, index 3, attention 1
+    assert layer.launches_per_step(_plan(3)) == 26
     # 128K mixed layer: the same kernels as the 1M layer (one attention launch for all heads)
-    assert layer.launches_per_step(_plan(2)) == 30
+    assert layer.launches_per_step(_plan(2)) == 29
     # one attention launch per pattern instead
-    assert layer.launches_per_step(_plan(2), fused=False) == 32
+    assert layer.launches_per_step(_plan(2), fused=False) == 31
 
 
 def test_digest_ignores_comments_and_whitespace():
