@@ -345,6 +345,45 @@ def mask_bs(rows, N: int, blk_idx, blk_cnt, block: int = 64) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# Grid pattern (MMInference abstract: video locality gives a Grid pattern,
+# handled through a permutation; the pages define no more, the reading is
+# stated in the design notes)
+# --------------------------------------------------------------------------
+
+def grid_select(q: np.ndarray, k: np.ndarray, P: int, scale: float, k_b: int, block: int = 64):
+    """Selection of a Grid head over a video segment of F frames x P tokens
+    per frame, tokens frame-major (i = f * P + p).  Reading: the tokens of one
+    in-frame position p, taken in frame order (rows p, p + P, p + 2P, ...),
+    form a sequence of their own, and each such sequence gets the
+    Block-Sparse selection (64-frame mean-pooled blocks, top-k_b per query
+    block, diagonal forced).  Returns idx [P, F/64, k_b] and cnt [P, F/64]."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    idx, cnt = [], []
+    for p in range(P):
+        i_, c_ = bs_select(q[p::P], k[p::P], scale, k_b, block)
+        idx.append(i_)
+        cnt.append(c_)
+    return np.stack(idx), np.stack(cnt)
+
+
+def mask_grid(rows, N: int, P: int, blk_idx, blk_cnt, block: int = 64) -> np.ndarray:
+    """Grid: key j is kept for query i when both sit at the same in-frame
+    position (j = i mod P), j <= i, and the 64-frame block of j's frame is
+    selected for the block of i's frame in that position's sequence."""
+    rows = np.asarray(rows)
+    j = np.arange(N)
+    out = np.zeros((rows.size, N), bool)
+    for r, i in enumerate(rows):
+        p, f = i % P, i // P
+        sel = np.zeros(N // P // block, bool)
+        b = f // block
+        sel[np.asarray(blk_idx[p][b][: int(blk_cnt[p][b])], np.int64)] = True
+        out[r] = (j <= i) & (j % P == p) & sel[(j // P) // block]
+    return out
+
+
+# --------------------------------------------------------------------------
 # Masked softmax attention
 # --------------------------------------------------------------------------
 

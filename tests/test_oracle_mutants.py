@@ -214,6 +214,31 @@ def _kept_mass_variant(q_rows, k, rows, mask, scale, *, over_mask=False, noncaus
     return np.where(keep, e, 0.0).sum(axis=1) / den
 
 
+def _grid_select_contiguous(q, k, P, scale, k_b, block=64):
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    F = q.shape[0] // P
+    idx, cnt = [], []
+    for p in range(P):
+        i_, c_ = _ORIG["bs_select"](q[p * F:(p + 1) * F], k[p * F:(p + 1) * F], scale, k_b, block)
+        idx.append(i_)
+        cnt.append(c_)
+    return np.stack(idx), np.stack(cnt)
+
+
+def _mask_grid_any_position(rows, N, P, blk_idx, blk_cnt, block=64):
+    rows = np.asarray(rows)
+    j = np.arange(N)
+    out = np.zeros((rows.size, N), bool)
+    for r, i in enumerate(rows):
+        p, f = i % P, i // P
+        sel = np.zeros(N // P // block, bool)
+        b = f // block
+        sel[np.asarray(blk_idx[p][b][: int(blk_cnt[p][b])], np.int64)] = True
+        out[r] = (j <= i) & sel[(j // P) // block]
+    return out
+
+
 def _to_f64_via_half(x):
     import torch
     if isinstance(x, torch.Tensor):
@@ -261,6 +286,8 @@ MUTANTS = {
     "to_f64: converted through float16": {"to_f64": _to_f64_via_half},
     "kept_mass: normalised over the mask": {
         "kept_mass": lambda q, k, r, m, sc: _kept_mass_variant(q, k, r, m, sc, over_mask=True)},
+    "grid_select: positions taken as contiguous runs": {"grid_select": _grid_select_contiguous},
+    "mask_grid: other in-frame positions kept": {"mask_grid": _mask_grid_any_position},
     "kept_mass: keys past the row counted": {
         "kept_mass": lambda q, k, r, m, sc: _kept_mass_variant(q, k, r, m, sc, noncausal=True)},
 }

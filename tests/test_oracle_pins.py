@@ -515,3 +515,60 @@ def test_kept_mass_equals_lse_ratio():
     _, lse_s = orc.attention_rows(q, k, v, mask, sc)
     _, lse_d = orc.attention_rows(q, k, v, causal, sc)
     np.testing.assert_allclose(orc.kept_mass(q, k, rows, mask, sc), np.exp(lse_s - lse_d), rtol=1e-12)
+
+
+# ---------------------------------------------------------------- Grid pattern
+def test_grid_with_one_position_is_block_sparse():
+    """P = 1: every token is at the same in-frame position, and the Grid
+    selection and mask are the Block-Sparse ones."""
+    rng = np.random.default_rng(8)
+    N, d = 512, 8
+    q, k = rng.normal(size=(N, d)), rng.normal(size=(N, d))
+    gi, gc = orc.grid_select(q, k, 1, 0.3, 3)
+    bi, bc = orc.bs_select(q, k, 0.3, 3)
+    assert np.array_equal(gi[0], bi) and np.array_equal(gc[0], bc)
+    rows = np.array([0, 70, 200, 511])
+    assert np.array_equal(orc.mask_grid(rows, N, 1, gi, gc), orc.mask_bs(rows, N, bi, bc))
+
+
+def test_grid_mask_bruteforce_loops():
+    """Plain loops over (i, j) with the position, causal and block rules."""
+    rng = np.random.default_rng(9)
+    P, F, d = 3, 256, 4
+    N = P * F
+    q, k = rng.normal(size=(N, d)), rng.normal(size=(N, d))
+    gi, gc = orc.grid_select(q, k, P, 0.5, 2)
+    rows = np.array([0, 2, 5, 190, 383, 600, N - 1])
+    got = orc.mask_grid(rows, N, P, gi, gc)
+    for r, i in enumerate(rows):
+        for j in range(N):
+            want = False
+            if j <= i and j % P == i % P:
+                sel = set(int(x) for x in gi[i % P][(i // P) // 64][: gc[i % P][(i // P) // 64]])
+                want = ((j // P) // 64) in sel
+            assert got[r, j] == want, (i, j)
+
+
+def test_grid_selection_follows_each_position_sequence():
+    """A block pair planted in one position's sequence is selected there and
+    not at the other positions; with every block selected the mask is every
+    earlier same-position key."""
+    rng = np.random.default_rng(10)
+    P, F, d = 2, 512, 8
+    N = P * F
+    q = rng.normal(size=(N, d)) * 0.1
+    k = rng.normal(size=(N, d)) * 0.1
+    u = np.zeros(d)
+    u[0] = 5.0
+    # position 1: query block 7 and key block 2 of its frame sequence share a direction
+    q[[f * P + 1 for f in range(7 * 64, 8 * 64)]] += u
+    k[[f * P + 1 for f in range(2 * 64, 3 * 64)]] += u
+    gi, gc = orc.grid_select(q, k, P, 1.0, 2)
+    assert 2 in gi[1][7][: gc[1][7]]
+    assert 2 not in gi[0][7][: gc[0][7]]
+    ai, ac = orc.grid_select(q, k, P, 1.0, F // 64)
+    rows = np.array([5, 700, N - 1])
+    m = orc.mask_grid(rows, N, P, ai, ac)
+    j = np.arange(N)
+    for r, i in enumerate(rows):
+        assert np.array_equal(m[r], (j <= i) & (j % P == i % P))
