@@ -13,7 +13,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["api.cu", "attn.cu", "bs_select.cu", "estimate.cu", "estimate_tc.cu", "index.cu", "noalloc.cu", "selftest.cu"]
+SOURCES = ["api.cu", "attn.cu", "bs_select.cu", "estimate.cu", "estimate_tc.cu", "grid.cu", "index.cu", "noalloc.cu",
+           "selftest.cu"]
 LIB = os.path.join(HERE, "libminf.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 

@@ -147,6 +147,41 @@ size_t plan_bs_est(const minf_shape* s, int nh, int k_b, char* ws, BsEstWs* out)
 // 3-D bf16 view of the split key means [3 * bh, nb, d]: x = d, y = key block,
 // z = part * bh + slot, with 64 x 128 x 1 boxes (128-byte swizzled); rows
 // past nb read as zero.
+// The Grid workspace: the Block-Sparse estimation's workspace of the permuted
+// shape first (its status block is the call's), then the permuted Q, K, V
+// and O, the permuted LSE and the selection (when the caller passes none).
+struct GridWs {
+  char* est;
+  size_t est_bytes;
+  __nv_bfloat16 *qp, *kp, *vp, *op;
+  float* lsep;
+  int32_t *bi, *bc;
+};
+minf_shape grid_shape(const minf_shape* s, int P) {
+  minf_shape g = *s;
+  g.B = s->B * P;
+  g.N = s->N / P;
+  return g;
+}
+size_t plan_grid(const minf_shape* s, int nh, int k_b, int P, char* ws, GridWs* out) {
+  const minf_shape g = grid_shape(s, P);
+  GridWs w;
+  w.est = ws;
+  w.est_bytes = plan_bs_est(&g, nh, k_b, nullptr, nullptr);
+  Carver c{ws, w.est_bytes};
+  const size_t rows_q = (size_t)s->B * s->Hq * s->N, rows_kv = (size_t)s->B * s->Hkv * s->N;
+  w.qp = c.take<__nv_bfloat16>(rows_q * s->d);
+  w.kp = c.take<__nv_bfloat16>(rows_kv * s->d);
+  w.vp = c.take<__nv_bfloat16>(rows_kv * s->d);
+  w.op = c.take<__nv_bfloat16>(rows_q * s->d);
+  w.lsep = c.take<float>(rows_q);
+  const size_t blocks = (size_t)g.B * nh * (g.N / 64);
+  w.bi = c.take<int32_t>(blocks * (size_t)std::max(k_b, 1));
+  w.bc = c.take<int32_t>(blocks);
+  if (out) *out = w;
+  return c.off;
+}
+
 // 3-D fp32 view of the pooled score matrices [bh, nb, nb]: x = key block,
 // y = query block, z = slot, with 32 x 128 x 1 boxes (128-byte swizzled).
 bool make_scores_map(CUtensorMap* m, const void* ptr, long long bh, int nb) {
@@ -270,6 +305,8 @@ size_t minf_workspace_size(int op, const minf_shape* s, int nh, int k_v, int k_s
     case MINF_OP_DENSE_ATTN:
     case MINF_OP_SPARSE_ATTN_LAYER:
       return kStatusBytes;
+    case MINF_OP_ATTN_GRID:
+      return plan_grid(s, nh, k_b, 1, nullptr, nullptr);  // one token per frame needs the most
     default:
       return 0;
   }
@@ -395,6 +432,70 @@ minf_status minf_estimate_bs(const minf_shape* s, const minf_bf16* Q, const minf
   t.status = w.status;
   t.scratch = nullptr;
   return cuda_status(topk_rows_launch(t, cs));
+}
+
+minf_status minf_attn_grid(const minf_shape* s, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
+                           const int32_t* heads, int nh, int frame_tokens, int k_b, int32_t* blk_idx,
+                           int32_t* blk_cnt, minf_bf16* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  minf_status st = check_shape(s);
+  if (st != MINF_OK) return st;
+  if (!Q || !K || !V || !heads || !O || !ws || nh < 1 || nh > s->Hq || k_b < 1) return MINF_ERR_INVALID_ARG;
+  const int P = frame_tokens;
+  if (P < 1 || s->N % P != 0 || (s->N / P) % 128 != 0) return MINF_ERR_INVALID_ARG;
+  if (((uintptr_t)Q | (uintptr_t)K | (uintptr_t)V | (uintptr_t)O) & 15) return MINF_ERR_INVALID_ARG;
+  if (ws_bytes < plan_grid(s, nh, k_b, P, nullptr, nullptr)) return MINF_ERR_WORKSPACE_TOO_SMALL;
+  GridWs w;
+  plan_grid(s, nh, k_b, P, (char*)ws, &w);
+  const minf_shape g = grid_shape(s, P);
+  int32_t* bi = blk_idx ? blk_idx : w.bi;
+  int32_t* bc = blk_cnt ? blk_cnt : w.bc;
+  cudaStream_t cs = (cudaStream_t)stream;
+  GridPermParams gp;
+  gp.B = s->B;
+  gp.N = s->N;
+  gp.F = s->N / P;
+  gp.P = P;
+  gp.d = s->d;
+  gp.status = reinterpret_cast<DevStatus*>(ws);
+  gp.dir = 0;
+  gp.lse_src = nullptr;
+  gp.lse_dst = nullptr;
+  // the listed heads' Q rows and every KV head's K and V rows, position-major
+  gp.src = reinterpret_cast<const __nv_bfloat16*>(Q);
+  gp.dst = w.qp;
+  gp.heads = heads;
+  gp.nh = nh;
+  gp.H = s->Hq;
+  if (grid_permute_launch(gp, cs) != cudaSuccess) return MINF_ERR_CUDA;
+  gp.heads = nullptr;
+  gp.nh = s->Hkv;
+  gp.H = s->Hkv;
+  gp.src = reinterpret_cast<const __nv_bfloat16*>(K);
+  gp.dst = w.kp;
+  if (grid_permute_launch(gp, cs) != cudaSuccess) return MINF_ERR_CUDA;
+  gp.src = reinterpret_cast<const __nv_bfloat16*>(V);
+  gp.dst = w.vp;
+  if (grid_permute_launch(gp, cs) != cudaSuccess) return MINF_ERR_CUDA;
+  // Block-Sparse estimation and attention on the B * P position sequences;
+  // both share the call's status block (at the workspace's start)
+  const minf_bf16* qp = reinterpret_cast<const minf_bf16*>(w.qp);
+  const minf_bf16* kp = reinterpret_cast<const minf_bf16*>(w.kp);
+  const minf_bf16* vp = reinterpret_cast<const minf_bf16*>(w.vp);
+  st = minf_estimate_bs(&g, qp, kp, heads, nh, 64, k_b, bi, bc, nullptr, w.est, w.est_bytes, stream);
+  if (st != MINF_OK) return st;
+  st = minf_sparse_attn_bs(&g, qp, kp, vp, heads, nh, bi, bc, k_b, reinterpret_cast<minf_bf16*>(w.op),
+                           lse ? w.lsep : nullptr, ws, kStatusBytes, stream);
+  if (st != MINF_OK) return st;
+  // the output (and LSE) rows back to frame-major order
+  gp.dir = 1;
+  gp.src = w.op;
+  gp.dst = reinterpret_cast<__nv_bfloat16*>(O);
+  gp.heads = heads;
+  gp.nh = nh;
+  gp.H = s->Hq;
+  gp.lse_src = lse ? w.lsep : nullptr;
+  gp.lse_dst = lse;
+  return cuda_status(grid_permute_launch(gp, cs));
 }
 
 minf_status minf_build_index(const minf_shape* s, int nh, const int32_t* v_idx, int k_v, const int32_t* s_idx,

@@ -136,6 +136,20 @@ bool bs_select_supported(int N, int d, int k);
 cudaError_t bs_select_launch(const CUtensorMap& tmKs, const CUtensorMap& tmS, const BsEstParams& p, int k,
                              int32_t* blk_idx, int32_t* blk_cnt, cudaStream_t stream);
 
+// Grid pattern row permutation (grid.cu): dir 0 gathers frame-major rows
+// [B, H, F * P, d] into position-major [B * P, H, F, d], dir 1 scatters back;
+// only the listed heads' rows (heads NULL: 0 .. nh-1); lse rows follow when set.
+struct GridPermParams {
+  const __nv_bfloat16* src;
+  __nv_bfloat16* dst;
+  const float* lse_src;
+  float* lse_dst;
+  const int32_t* heads;
+  int nh, B, H, N, F, P, d, dir;
+  DevStatus* status;
+};
+cudaError_t grid_permute_launch(const GridPermParams& p, cudaStream_t stream);
+
 struct VsIndexParams {
   const int32_t* v_idx;
   const int32_t* s_idx;

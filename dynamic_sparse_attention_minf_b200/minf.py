@@ -19,13 +19,14 @@ OK = 0
 STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error",
                 4: "workspace too small", 5: "device timeout", 6: "device bounds"}
 OP_ESTIMATE_VS, OP_ESTIMATE_BS, OP_BUILD_INDEX, OP_SPARSE_ATTN_VS, OP_SPARSE_ATTN_BS, \
-    OP_ATTN_ASHAPE, OP_DENSE_ATTN, OP_BUILD_INDEX_EXACT, OP_SPARSE_ATTN_VS_EXACT, OP_SPARSE_ATTN_LAYER = range(10)
+    OP_ATTN_ASHAPE, OP_DENSE_ATTN, OP_BUILD_INDEX_EXACT, OP_SPARSE_ATTN_VS_EXACT, OP_SPARSE_ATTN_LAYER, \
+    OP_ATTN_GRID = range(11)
 
 EXPORTS = ["minf_vs_wmap_words", "minf_workspace_size", "minf_estimate_vs", "minf_estimate_bs",
            "minf_build_index", "minf_sparse_attn_vs", "minf_sparse_attn_bs", "minf_attn_ashape",
            "minf_dense_attn", "minf_get_device_status", "minf_status_string", "minf_vs_bits_words",
            "minf_vs_twmap_words", "minf_build_index_exact", "minf_sparse_attn_vs_exact",
-           "minf_sparse_attn_layer", "minf_selftest_exp2"]
+           "minf_sparse_attn_layer", "minf_selftest_exp2", "minf_attn_grid"]
 
 
 class MinfError(RuntimeError):
@@ -84,6 +85,7 @@ def lib():
         L.minf_selftest_exp2.argtypes = [vp, vp, vp, i, vp]
         L.minf_sparse_attn_layer.argtypes = [sp, vp, vp, vp, vp, i, ctypes.POINTER(_VsIndexC), i, i, vp, i, vp,
                                              vp, i, vp, i, i, i, vp, vp, vp, sz, vp]
+        L.minf_attn_grid.argtypes = [sp, vp, vp, vp, vp, i, i, i, vp, vp, vp, vp, vp, sz, vp]
         L.minf_get_device_status.argtypes = [vp, vp]
         L.minf_status_string.argtypes = [st]
         L.minf_status_string.restype = ctypes.c_char_p
@@ -333,6 +335,30 @@ def minf_dense_attn(q, k, v, heads=None, o=None, lse=None, want_lse=True, scale=
         ctypes.byref(shp), _p(q), _p(k), _p(v), _p(hd), nh, _p(o), _p(lse), _p(ws), ws.numel(),
         _stream(stream)))
     return o, lse
+
+
+def minf_attn_grid(q, k, v, heads, frame_tokens, k_b, o=None, lse=None, want_lse=True, scale=0.0,
+                   return_selection=False, ws=None, stream=None):
+    """Grid-pattern attention (see include/minf.h): the Block-Sparse
+    treatment of each in-frame position's frame sequence.  With
+    ``return_selection`` also returns blk_idx [B, P, nh, F/64, k_b] and
+    blk_cnt [B, P, nh, F/64]."""
+    shp = shape_of(q, k, scale)
+    hd = _heads(heads, q.device)
+    nh = hd.numel()
+    o, lse = _out(q, o, lse, want_lse)
+    P = int(frame_tokens)
+    bi = bc = None
+    if return_selection:
+        nbf = shp.N // P // 64
+        bi = torch.empty(shp.B, P, nh, nbf, k_b, dtype=torch.int32, device=q.device)
+        bc = torch.empty(shp.B, P, nh, nbf, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = workspace(OP_ATTN_GRID, shp, nh, k_b=k_b, device=q.device)
+    _check("minf_attn_grid", lib().minf_attn_grid(
+        ctypes.byref(shp), _p(q), _p(k), _p(v), _p(hd), nh, P, k_b, _p(bi), _p(bc), _p(o), _p(lse),
+        _p(ws), ws.numel(), _stream(stream)))
+    return (o, lse, bi, bc) if return_selection else (o, lse)
 
 
 def minf_sparse_attn_layer(q, k, v, vs_heads=None, vs_index: VSIndex | None = None, bs_heads=None,

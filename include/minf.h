@@ -327,7 +327,7 @@ enum { MINF_OP_SPARSE_ATTN_LAYER = 9 };
 /*
  * Attention of every head of a layer whose heads follow different patterns
  * (summary page, "Summary": a pattern per head, chosen offline; attention over
- * the estimated indices only), in one persistent launch: the Vertical-Slash
+ * the estimated indices only), in one launch: the Vertical-Slash
  * heads vs_heads[n_vs] with the index vs_idx (as minf_sparse_attn_vs), the
  * Block-Sparse heads bs_heads[n_bs] with blk_idx / blk_cnt (as
  * minf_sparse_attn_bs) and the A-shape heads a_heads[n_a] (as
@@ -368,6 +368,35 @@ minf_status minf_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int
 
 /* Static description of a status code. */
 const char* minf_status_string(minf_status s);
+
+/* ---------------------------------------------------------------------------
+ * Grid pattern (MMInference abstract: the temporal and spatial locality of
+ * video gives a Grid pattern, handled through a permutation).
+ * ------------------------------------------------------------------------- */
+enum { MINF_OP_ATTN_GRID = 10 };
+
+/*
+ * Grid-pattern attention of the listed heads over a video segment of
+ * N / frame_tokens frames of frame_tokens tokens each, stored frame-major
+ * (token i = f * frame_tokens + p).  Reading (the abstract defines no more):
+ * a query attends to keys at its own in-frame position p; the tokens of one
+ * position, in frame order, form a sequence of their own, and each such
+ * sequence gets the Block-Sparse treatment of minf_estimate_bs and
+ * minf_sparse_attn_bs (64-frame mean-pooled blocks, the k_b best key blocks
+ * per query block, the diagonal block forced, causal in frame order, which
+ * is causal in token order).  Implemented as that permutation: the rows are
+ * gathered position-major into the workspace, the two Block-Sparse calls run
+ * on the shape (B * frame_tokens, Hq, Hkv, N / frame_tokens, d), and O (and
+ * lse) are scattered back to the listed heads' rows.  N / frame_tokens must
+ * be a multiple of 128.  blk_idx [B, frame_tokens, nh, N / frame_tokens / 64,
+ * k_b] and blk_cnt [B, frame_tokens, nh, N / frame_tokens / 64] receive the
+ * per-position selections when non-NULL (the workspace holds them
+ * otherwise).  Workspace: minf_workspace_size(MINF_OP_ATTN_GRID, shape, nh,
+ * 0, 0, k_b), which covers every frame_tokens.
+ */
+minf_status minf_attn_grid(const minf_shape* shape, const minf_bf16* Q, const minf_bf16* K, const minf_bf16* V,
+                           const int32_t* heads, int nh, int frame_tokens, int k_b, int32_t* blk_idx,
+                           int32_t* blk_cnt, minf_bf16* O, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }
