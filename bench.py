@@ -547,7 +547,9 @@ def run_kernel_case(args):
     workload's budgets, vertical 2000 / slash 12000).  The index is built
     once; then the kernel runs ``--warmup`` + ``--steps`` times.
     ``--kernel vs_est|bs_est`` runs the index estimation of those 8 heads
-    instead (vertical 2000 / slash 12000; top-100 blocks)."""
+    instead (vertical 2000 / slash 12000; top-100 blocks), and ``--kernel grid``
+    the Grid-pattern attention of the 8 heads over ``--N`` / 256 frames of 256
+    tokens (top-100 frame blocks), timed with CUDA events."""
     from dynamic_sparse_attention_minf_b200 import layer, minf
     from dynamic_sparse_attention_minf_b200 import workloads as wl
     w = wl.config(WORKLOAD_ID, N=args.N)
@@ -555,6 +557,30 @@ def run_kernel_case(args):
     w.patterns = [wl.PAT_VS] * 8
     q, k, v = wl.make_qkv(w, "cuda")
     o = torch.empty_like(q)
+    if args.kernel == "grid":
+        shp = minf.shape_of(q, k)
+        heads = list(range(8))
+        P, k_b = 256, 100
+        ws = minf.workspace(minf.OP_ATTN_GRID, shp, 8, k_b=k_b)
+        fn = lambda: minf.minf_attn_grid(q, k, v, heads, P, k_b, o=o, want_lse=False, ws=ws)
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ws.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        tiles, nnz = _counters(ws)
+        # permutation traffic: Q and O of the 8 heads and K and V of the 2 KV heads, read and written
+        perm_bytes = 2 * (2 * 8 + 2 * 2) * w.N * w.d * 2
+        print(json.dumps({"kernel": "grid", "N": args.N, "frame_tokens": P, "frames": args.N // P, "k_b": k_b,
+                          "ms": ms, "tiles_per_call": tiles // args.steps, "useful_tflop": 4.0 * w.d * nnz / args.steps / 1e12,
+                          "permuted_bytes": perm_bytes, "status": minf.minf_get_device_status(ws)}))
+        return
     if args.kernel in ("vs_est", "bs_est"):
         shp = minf.shape_of(q, k)
         heads = list(range(8))
@@ -604,7 +630,7 @@ def main():
     ap.add_argument("--config", type=int, default=WORKLOAD_ID, choices=[2, 3, 4],
                     help="workload: 4 (default) the 1M-token mixed layer, 2 the 128K mixed layer, "
                          "3 the 512K all-Vertical-Slash layer")
-    ap.add_argument("--kernel", choices=["dense", "vs", "vs_est", "bs_est"], default=None,
+    ap.add_argument("--kernel", choices=["dense", "vs", "vs_est", "bs_est", "grid"], default=None,
                     help="run only this attention kernel on a small case (for profiling)")
     ap.add_argument("--N", type=int, default=262144, help="tokens of the --kernel case")
     ap.add_argument("--shard", choices=["kv", "replicas"], default="kv",
