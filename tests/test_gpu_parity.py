@@ -189,7 +189,7 @@ def _bs_pipeline(w, heads, rows=None):
     return flips
 
 
-@pytest.mark.parametrize("N,d", [(2048, 128), (640, 128), (1152, 64)])
+@pytest.mark.parametrize("N,d", [(2048, 128), (640, 128), (1152, 64), (8448, 128)])
 def test_bs_pipeline_small(N, d):
     w = wl.small(Hq=4, Hkv=2, N=N, d=d, seed=4, bias="block", patterns=[wl.PAT_BS] * 4, k_b=7)
     _bs_pipeline(w, [1, 2])
