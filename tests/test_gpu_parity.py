@@ -275,6 +275,39 @@ def test_minimum_size_one_tile(d):
     _check_attn(o, lse, qn, kn, vn, [0, 1], w, lambda hi, h: (lambda r: orc.mask_dense(r, w.N)))
 
 
+@pytest.mark.parametrize("last_q,d", [(1, 64), (17, 128), (32, 64), (64, 128)])
+def test_vs_estimation_last_rows(last_q, d):
+    """Fewer than 64 scoring rows: the rows before the last `last_q` are masked
+    in both passes, scores and sets match the oracle fed only those rows."""
+    N = 1280
+    w = wl.small(Hq=4, Hkv=2, N=N, d=d, seed=36, k_v=100, k_s=200)
+    q, k, v, qn, kn, vn = _inputs(w)
+    sc = orc.default_scale(d)
+    heads = [3, 0]
+    ws = minf.workspace(minf.OP_ESTIMATE_VS, minf.shape_of(q, k), 2)
+    v_idx, s_idx, vs, ss = minf.minf_estimate_vs(q, k, heads, w.k_v, w.k_s, last_q=last_q,
+                                                 return_scores=True, ws=ws)
+    assert minf.minf_get_device_status(ws) == 0
+    gv, gs = v_idx[0].cpu().numpy(), s_idx[0].cpu().numpy()
+    for hi, h in enumerate(heads):
+        kv = orc.kv_head(h, w.Hq, w.Hkv)
+        rv, rs = orc.vs_estimate(qn[h][N - last_q:], kn[kv], sc)
+        np.testing.assert_allclose(vs[0, hi].cpu().numpy(), rv, rtol=1e-4, atol=1e-7)
+        np.testing.assert_allclose(ss[0, hi].cpu().numpy(), rs, rtol=1e-4, atol=1e-7)
+        ov, os_ = orc.vs_select(rv, rs, w.k_v, w.k_s)
+        check_index_set(gv[hi], ov, rv, what=f"vertical h{h}")
+        check_index_set(gs[hi], os_, rs, forced=0, what=f"slash h{h}")
+
+
+def test_vs_estimation_bit_reproducible():
+    """Fixed-order sums: two runs give identical scores, bit for bit."""
+    w = wl.small(Hq=2, Hkv=1, N=4096, d=128, seed=37)
+    q, k, v = wl.make_qkv(w, DEV)
+    runs = [minf.minf_estimate_vs(q, k, [0, 1], 300, 600, return_scores=True) for _ in range(2)]
+    for a, b in zip(runs[0], runs[1]):
+        assert torch.equal(a, b)
+
+
 @pytest.mark.parametrize("N,k_v,k_s", [(65536, 1000, 3000), (131072, 2000, 6000)])
 def test_vs_estimation_long_rows(N, k_v, k_s):
     """Rows longer than 32K take the many-CTA top-k (several segments per row)."""
