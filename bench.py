@@ -549,9 +549,33 @@ def run_kernel_case(args):
     ``--kernel vs_est|bs_est`` runs the index estimation of those 8 heads
     instead (vertical 2000 / slash 12000; top-100 blocks), and ``--kernel grid``
     the Grid-pattern attention of the 8 heads over ``--N`` / 256 frames of 256
-    tokens (top-100 frame blocks), timed with CUDA events."""
+    tokens (top-100 frame blocks), timed with CUDA events.  ``--kernel
+    vs_est_layer`` times the Vertical-Slash estimation of all VS heads of the
+    ``--config`` layer at full size."""
     from dynamic_sparse_attention_minf_b200 import layer, minf
     from dynamic_sparse_attention_minf_b200 import workloads as wl
+    if args.kernel == "vs_est_layer":
+        # Vertical-Slash estimation of every VS head of the --config layer at
+        # its full size, 3 rounds of one untimed and 5 timed calls (CUDA events)
+        w = wl.config(args.config)
+        q, k, v = wl.make_qkv(w, "cuda")
+        heads = w.heads_of(wl.PAT_VS)
+        ws = minf.workspace(minf.OP_ESTIMATE_VS, minf.shape_of(q, k), len(heads))
+        out, res = None, []
+        for _ in range(3):
+            minf.minf_estimate_vs(q, k, heads, w.k_v, w.k_s, ws=ws)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(5):
+                out = minf.minf_estimate_vs(q, k, heads, w.k_v, w.k_s, ws=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            res.append(round(e0.elapsed_time(e1) / 5, 3))
+        print(json.dumps({"kernel": args.kernel, "workload": w.name, "N": w.N, "heads": len(heads),
+                          "vs_est_ms": res, "status": minf.minf_get_device_status(ws),
+                          "v_sum": int(out[0].sum().item()), "s_sum": int(out[1].sum().item())}))
+        return
     w = wl.config(WORKLOAD_ID, N=args.N)
     w.Hq, w.Hkv = 8, 2
     w.patterns = [wl.PAT_VS] * 8
@@ -630,8 +654,9 @@ def main():
     ap.add_argument("--config", type=int, default=WORKLOAD_ID, choices=[2, 3, 4],
                     help="workload: 4 (default) the 1M-token mixed layer, 2 the 128K mixed layer, "
                          "3 the 512K all-Vertical-Slash layer")
-    ap.add_argument("--kernel", choices=["dense", "vs", "vs_est", "bs_est", "grid"], default=None,
-                    help="run only this attention kernel on a small case (for profiling)")
+    ap.add_argument("--kernel", choices=["dense", "vs", "vs_est", "bs_est", "grid", "vs_est_layer"], default=None,
+                    help="run only this kernel on a small case (for profiling); vs_est_layer times the "
+                         "Vertical-Slash estimation of the --config layer's VS heads at full size")
     ap.add_argument("--N", type=int, default=262144, help="tokens of the --kernel case")
     ap.add_argument("--shard", choices=["kv", "replicas"], default="kv",
                     help="with several GPUs: split one layer by KV-head group (default) or run a layer per rank")
