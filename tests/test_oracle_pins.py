@@ -211,6 +211,20 @@ def test_vs_estimate_mass_closed_form():
     assert v[N - 1] < 1.0
 
 
+def test_vs_estimate_single_last_row():
+    """One scoring row (the last, i = N - 1): v is that row's softmax and the
+    slash score of offset o is the entry of key N - 1 - o, so sigma is v
+    reversed; the softmax itself is scipy's."""
+    from scipy.special import softmax
+    rng = np.random.default_rng(5)
+    N, d = 300, 16
+    q, k = rng.standard_normal((1, d)), rng.standard_normal((N, d))
+    sc = 1 / math.sqrt(d)
+    v, sg = orc.vs_estimate(q, k, sc)
+    assert np.allclose(v, softmax(sc * (k @ q[0])), atol=1e-14)
+    assert np.allclose(sg, v[::-1], atol=1e-14)
+
+
 def test_vs_planted_column_and_diagonal():
     rng = np.random.default_rng(9)
     N, d = 1024, 32
